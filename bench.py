@@ -1,0 +1,379 @@
+"""Benchmark of the GPTQ layer solver (Hessian + prepare + sweep + pack per layer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload opt125m]
+
+One step quantizes every layer of the workload once: Hessian accumulation over
+all calibration tokens, damping / ordering / inverse Cholesky factor, the
+blocked column sweep, and bit packing.  Inputs are seeded synthetic tensors
+resident in HBM before timing; the calibration set (2.4 GB for the default
+workload) is larger than L2, so no flush is needed between steps.
+
+Multi-GPU: one process per GPU (torchrun).  The path has no exchange step, so
+every rank quantizes its own replica of the workload (weak scaling); the only
+collectives are the timing barrier and the max-over-ranks of the elapsed time.
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from post_weight_quantization_20_b200 import synthetic as S  # noqa: E402
+from post_weight_quantization_20_b200.workloads import WORKLOADS  # noqa: E402
+
+METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200 peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+def workload_config(wl, n_gpus):
+    shapes = ", ".join(f"{l.rows}x{l.cols}" for l in wl.layers)
+    q = wl.quant[0]
+    return {
+        "workload": f"{wl.name}: W {shapes} {wl.wdtype}; X {wl.tokens} tokens x cols {wl.xdtype} "
+                    f"({wl.xspec.dist}, {wl.xspec.outlier_frac:.0%} outlier channels x{wl.xspec.outlier_mult:g}); "
+                    f"{q.label()} B={q.block_size} damp={q.damp}",
+        "layers": len(wl.layers),
+        "calib_tokens": wl.tokens,
+        "l2": "inputs larger than L2 (calibration set > 126 MB), no flush",
+        "parallelism": f"replicas x{n_gpus} (no data-path collective)",
+    }
+
+
+def gen_inputs(wl, seed=1234):
+    out = []
+    for l in wl.layers:
+        W = S.gen_weight(l.rows, l.cols, wl.wdtype, wl.wspec, seed=seed, tag=l.tag)
+        X = S.gen_activations(wl.tokens, l.cols, wl.xdtype, wl.xspec, seed=seed, tag=l.tag)
+        out.append((l, W, X))
+    return out
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    from post_weight_quantization_20_b200 import gptq as G
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    G.load_library()
+    wl = WORKLOADS[args.workload]
+    q = wl.quant[0]
+    cfg = G.make_config(q.bits, q.group_size, q.sym, q.act_order, q.damp, q.block_size)
+    host = gen_inputs(wl)
+    torch_dt = {S.F32: torch.float32, S.F16: torch.float16, S.BF16: torch.bfloat16}
+
+    def to_dev(a, dt):
+        if dt == S.BF16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    def to_pinned(a, dt):
+        t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if dt == S.BF16 else torch.from_numpy(a)
+        return t.pin_memory()
+
+    stream = torch.cuda.current_stream(dev)
+    layers = []
+    for l, W, X in host:
+        R, C = l.rows, l.cols
+        Gn = G.n_groups(C, cfg.group_size)
+        b = {
+            "R": R, "C": C,
+            "W": to_dev(W, wl.wdtype), "X": to_dev(X, wl.xdtype),
+            "H": torch.empty(C, C, device=dev), "U": torch.empty(C, C, device=dev),
+            "perm": torch.empty(C, dtype=torch.int32, device=dev),
+            "wsp": G.alloc_workspace(G.GPTQ_OP_PREPARE, R, C, cfg, dev),
+            "wsq": G.alloc_workspace(G.GPTQ_OP_QUANTIZE, R, C, cfg, dev),
+            "codes": torch.empty(R, C, dtype=torch.uint8, device=dev),
+            "scales": torch.empty(R, Gn, device=dev), "zeros": torch.empty(R, Gn, device=dev),
+            "g_idx": torch.empty(C, dtype=torch.int32, device=dev),
+            "losses": torch.empty(C, device=dev),
+            "packed": torch.empty(R, G.packed_words(C, cfg.bits), dtype=torch.int32, device=dev),
+            "status": torch.zeros(1, dtype=torch.int32, device=dev),
+        }
+        layers.append(b)
+
+    hess_ev = []
+
+    def step(record=False):
+        for b in layers:
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            G.gptq_hessian_accumulate(b["H"], 0, b["X"], b["status"], stream)
+            if record:
+                e1.record(stream)
+                hess_ev.append((e0, e1, b["X"].shape[0], b["C"]))
+            G.gptq_prepare(b["H"], cfg, b["U"], b["perm"], b["wsp"], b["status"], stream)
+            G.gptq_quantize_layer(b["W"], b["U"], b["perm"], cfg, b["codes"], b["scales"],
+                                  b["zeros"], b["g_idx"], b["losses"], b["wsq"], b["status"], stream)
+            G.gptq_pack(b["codes"], cfg.bits, b["packed"], stream)
+
+    import torch.distributed as dist
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    for b in layers:
+        st = int(b["status"].item())
+        if st:
+            raise RuntimeError(f"device status {G.status_names(st)}")
+
+    clocks = ClockSampler(local_rank)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    launches0 = G.gptq_launch_count()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = G.gptq_launch_count() - launches0
+    barrier()
+    cl = clocks.stop()
+    ms = t0.elapsed_time(t1)
+    hess_ms = sum(a.elapsed_time(b) for a, b, _, _ in hess_ev)
+    hess_flop = sum(float(m) * C * (C + 1) for _, _, m, C in hess_ev)
+    n_hess = len(hess_ev)
+
+    # end to end through the public API from pinned host buffers
+    pinned = [(l, to_pinned(W, wl.wdtype), to_pinned(X, wl.xdtype)) for l, W, X in host]
+    h2d = sum(w.numel() * w.element_size() + x.numel() * x.element_size() for _, w, x in pinned)
+
+    def e2e_step():
+        outs = []
+        for l, Wh, Xh in pinned:
+            r = G.quantize_layer_host(Wh, Xh, cfg, device=dev)
+            outs.append(r)
+        return outs
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    e2e_steps = max(1, min(args.steps, 5))
+    d2h = 0
+    for _ in range(e2e_steps):
+        outs = e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    d2h = sum(o.nbytes for o in outs)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    if world > 1:
+        t = torch.tensor([ms, e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(t[0]), float(t[1])
+
+    n_layers = len(layers) * world
+    peaks = load_peaks()
+    achieved = hess_flop / (hess_ms * 1e-3) / 1e12 if hess_ms > 0 else None
+    peak = float(peaks["bf16_tflops"])
+    out = {
+        "metric": METRIC,
+        "value": ms / args.steps / n_layers,
+        "unit": "ms",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms / args.steps,
+        "higher_is_better": False,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": f"{wl.xdtype} inputs, f32 accumulate/solve",
+        "data": "synthetic (seeded; stands in for the pages' calibration text)",
+        "config": workload_config(wl, world),
+        "hessian": {"ms_per_launch": hess_ms / max(n_hess, 1), "tflops": achieved,
+                    "launches": n_hess},
+        "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 dense burst"},
+        "e2e": {"value": e2e_ms / len(layers), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": int(launches),
+        "clocks": cl,
+    }
+    return out
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_layer(W, X, wl, q):
+    from oracle import gptq_ref as o
+    X64 = S.to_f64(X, wl.xdtype)
+    H, n = o.hessian(X64)
+    del X64
+    out = o.gptq_quantize(S.to_f64(W, wl.wdtype), H, q.bits, q.group_size, q.sym, q.act_order,
+                          q.damp, q.block_size)
+    o.pack(out["codes"], q.bits)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info if i.get("user_api") == "blas"] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_sample(wl):
+    """A bounded sample of the workload for the oracle: its first layer."""
+    l = wl.layers[0]
+    W = S.gen_weight(l.rows, l.cols, wl.wdtype, wl.wspec, seed=1234, tag=l.tag)
+    X = S.gen_activations(wl.tokens, l.cols, wl.xdtype, wl.xspec, seed=1234, tag=l.tag)
+    return l, W, X
+
+
+def run_cpu_baseline(wl):
+    q = wl.quant[0]
+    l, W, X = cpu_sample(wl)
+    t = time.perf_counter()
+    oracle_layer(W, X, wl, q)
+    dt = time.perf_counter() - t
+    return {"value": dt * 1e3, "unit": "ms per layer", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one {l.rows}x{l.cols} layer ({l.name}) with all {wl.tokens} calibration tokens, "
+                      f"float64 NumPy oracle"}
+
+
+def run_reference(args):
+    wl = WORKLOADS[args.workload]
+    q = wl.quant[0]
+    l, W, X = cpu_sample(wl)
+    for _ in range(args.warmup):
+        oracle_layer(W, X, wl, q)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_layer(W, X, wl, q)
+    dt = (time.perf_counter() - t) / args.steps
+    v = dt * 1e3
+    cores = blas_threads()
+    sample = (f"one {l.rows}x{l.cols} layer ({l.name}) of the workload per step, all "
+              f"{wl.tokens} calibration tokens, float64 NumPy oracle on host cores")
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)", "config": workload_config(wl, 1),
+            "cpu_baseline": {"value": v, "unit": "ms per layer", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="opt125m", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = run_cpu_baseline(WORKLOADS[args.workload])
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,178 @@
+/*
+ * gptq.h — C ABI of libgptq.so, a B200 (sm_100a) GPTQ layer-wise quantization solver.
+ *
+ * The calls follow the per-layer flow of "GPTQ量化算法深度解析：从Hessian曲率到大模型单卡部署"
+ * (sheratonhq.com) §3.1: add calibration batches to the Hessian (step 1), factor it
+ * (step 2), sweep the columns in blocks with error feedback (step 3), store codes and
+ * quantization parameters (step 4).  Quantizer parameters (bits, group size, sym,
+ * desc_act, damp_percent) are those of §3.3 of the same page and of the table
+ * "bits、group_size、sym 与 desc_act 分别影响什么" of the lansai.wang deployment guide.
+ *
+ * Conventions shared by every call
+ *  - Array arguments are DEVICE pointers owned by the caller; the library never
+ *    allocates or frees device memory.  Scratch memory is the caller's `ws`
+ *    buffer, sized with gptq_workspace_size().
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Host-side results (n_seen) are updated
+ *    at enqueue time.
+ *  - Return value: GPTQ_OK, or exactly one error code.  Argument errors are
+ *    detected on the host before anything is launched.  GPTQ_ERR_CUDA means a
+ *    launch failed (cudaGetLastError() was not cudaSuccess).
+ *  - Conditions only the device can see are OR-ed as gptq_status bits into
+ *    `*dev_status` (a caller-owned device int32, may be NULL to ignore them):
+ *    GPTQ_ERR_NOT_PD (non-positive pivot), GPTQ_ERR_NONFINITE (NaN/Inf in H),
+ *    GPTQ_ERR_INVALID_ARG (a caller-supplied permutation is not a permutation),
+ *    GPTQ_ERR_TIMEOUT (a bounded device wait gave up).  Kernels never trap; the
+ *    caller reads *dev_status after synchronizing the stream.
+ *  - Matrices are row-major.  W is rows x cols (out x in features, as a PyTorch
+ *    Linear weight); X is tokens x cols.
+ */
+#ifndef GPTQ_H_
+#define GPTQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes.  Values are distinct bits so device conditions can be OR-ed. */
+typedef enum {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1,
+  GPTQ_ERR_UNSUPPORTED = 2,
+  GPTQ_ERR_WORKSPACE = 4,
+  GPTQ_ERR_NOT_PD = 8,
+  GPTQ_ERR_NONFINITE = 16,
+  GPTQ_ERR_TIMEOUT = 32,
+  GPTQ_ERR_CUDA = 64
+} gptq_status;
+
+/* Element types of W and X. */
+typedef enum { GPTQ_F32 = 0, GPTQ_F16 = 1, GPTQ_BF16 = 2 } gptq_dtype;
+
+/* act_order values. */
+enum { GPTQ_ORDER_NATURAL = 0, GPTQ_ORDER_DESC_DIAG = 1, GPTQ_ORDER_GIVEN = 2 };
+
+/* Workspace queries. */
+enum { GPTQ_OP_PREPARE = 1, GPTQ_OP_QUANTIZE = 2 };
+
+/*
+ * Quantizer configuration (GPTQ量化算法深度解析 §3.3; lansai.wang guide, parameter table).
+ *  bits        2, 3, 4 or 8: codes take values 0 .. 2^bits - 1.
+ *  group_size  0 (or -1): one grid per row, from the row before any compensation.
+ *              g > 0: one grid per g consecutive columns in sweep order, computed when
+ *              the sweep reaches the group's first column from the current compensated
+ *              weights.  g must divide 128 (the kernels' column panel).
+ *  sym         0: asymmetric min-max grid containing 0, integer zero-point
+ *              z = rint(-lo/s).  1: symmetric range [-max|v|, max|v|], z = 2^(bits-1).
+ *  act_order   GPTQ_ORDER_NATURAL, GPTQ_ORDER_DESC_DIAG (columns by descending
+ *              diag(H), ties by ascending index; "desc_act"), or GPTQ_ORDER_GIVEN
+ *              (perm supplied by the caller to gptq_prepare).
+ *  damp        relative damping: lambda = damp * mean(diag H) is added to diag H.
+ *  block_size  lazy-batch width B of §2.4.  Lazy batching is exact, so B changes
+ *              rounding only; the kernels always sweep 128-column panels.  Must be
+ *              >= 1, and group_size must divide B or be a multiple of it.
+ */
+typedef struct {
+  int bits;
+  int group_size;
+  int sym;
+  int act_order;
+  float damp;
+  int block_size;
+} gptq_config;
+
+/*
+ * gptq_workspace_size — bytes of `ws` needed by gptq_prepare (op = GPTQ_OP_PREPARE)
+ * or gptq_quantize_layer (op = GPTQ_OP_QUANTIZE) for the given shape.  Returns 0
+ * for invalid arguments.  The result is a multiple of 256.
+ */
+size_t gptq_workspace_size(int op, int64_t rows, int64_t cols, const gptq_config* cfg);
+
+/*
+ * gptq_hessian_accumulate — GPTQ量化算法深度解析 §3.1 step 1 (H = 2 X X^T, normalised).
+ * Adds a chunk of m calibration tokens to the running Hessian:
+ *     H <- H * n/(n+m) + (2/(n+m)) * X^T X,      n <- n + m
+ *  H        cols x cols fp32, row-major.  Only the upper triangle (i <= j) is read
+ *           and written; the strictly lower triangle is left untouched.  When
+ *           *n_seen == 0 the upper triangle is overwritten (need not be initialised).
+ *  n_seen   HOST pointer to the number of tokens already in H; updated on enqueue.
+ *  X        device pointer, m_tokens x cols, row stride ldx elements (ldx >= cols),
+ *           element type xdtype.  16-bit X with ldx a multiple of 8 and a 16-byte
+ *           aligned base runs on the tcgen05 tensor cores (fp32 accumulate).
+ *  dev_status  see conventions (may be NULL).
+ *  m_tokens == 0 is a no-op.  Errors: INVALID_ARG (null pointer, cols <= 0,
+ *  m_tokens < 0, ldx < cols, bad dtype).
+ */
+gptq_status gptq_hessian_accumulate(float* H, int64_t* n_seen, const void* X, int xdtype,
+                                    int64_t m_tokens, int64_t cols, int64_t ldx,
+                                    int32_t* dev_status, void* stream);
+
+/*
+ * gptq_prepare — GPTQ量化算法深度解析 §3.1 step 2 and §2.4 (Cholesky), §3.3 (damping,
+ * desc_act).  Reads the upper triangle of H, damps it by lambda = damp*mean(diag H),
+ * orders the columns, and writes the inverse Cholesky factor of the permuted matrix:
+ *     Hp = (H + lambda I)[perm][:, perm],     U upper triangular, U^T U = Hp^-1,
+ *     U[q][q] > 0, entries below the diagonal written as 0.
+ *  H     cols x cols fp32 (upper triangle used; not modified).
+ *  U     cols x cols fp32 output, row-major.
+ *  perm  cols int32: output for NATURAL / DESC_DIAG (perm[j] = original column
+ *        swept j-th); input for GIVEN (checked on the device: a bad permutation
+ *        sets GPTQ_ERR_INVALID_ARG in *dev_status).
+ *  ws    workspace of at least gptq_workspace_size(GPTQ_OP_PREPARE, 0, cols, cfg)
+ *        bytes, 256-byte aligned.
+ *  Device conditions: NONFINITE (diag(H) not finite), NOT_PD (a pivot <= 0; the
+ *  factor is then not meaningful).  Errors: INVALID_ARG, WORKSPACE.
+ */
+gptq_status gptq_prepare(const float* H, int64_t cols, const gptq_config* cfg, float* U,
+                         int32_t* perm, void* ws, size_t ws_bytes, int32_t* dev_status,
+                         void* stream);
+
+/*
+ * gptq_quantize_layer — GPTQ量化算法深度解析 §2.2 (OBS compensation), §2.4 (fixed order,
+ * lazy batch updates), §3.1 step 3-4.  Sweeps the columns of W in the order perm,
+ * 128 at a time.  For each column q (in sweep order), with d = U[q][q]:
+ *     code = clamp(rint(w/s) + z, 0, 2^bits-1),  Q = s (code - z),
+ *     err = (w - Q)/d,   w[q+1 : block end] -= err * U[q][q+1 : block end]
+ * and after each block  W[:, end:] -= Err * U[block, end:].
+ *  W       rows x cols, row stride ldw elements, element type wdtype; not modified.
+ *  U, perm as produced by gptq_prepare.
+ *  codes   rows x cols uint8, ORIGINAL column order.
+ *  scales, zeros  rows x G fp32, G = ceil(cols/group_size) (1 for per-row grids),
+ *          groups in sweep order; zeros hold integers.
+ *  g_idx   cols int32: group of each original column (0 for per-row grids).
+ *  losses  cols fp32: sum over rows of (w - Q)^2 / (2 d^2), ORIGINAL column order.
+ *  ws      at least gptq_workspace_size(GPTQ_OP_QUANTIZE, rows, cols, cfg) bytes.
+ *  rows == 0 writes only g_idx and zero losses.  Errors: INVALID_ARG,
+ *  UNSUPPORTED (group_size does not divide 128, or not compatible with block_size),
+ *  WORKSPACE.
+ */
+gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t cols,
+                                int64_t ldw, const float* U, const int32_t* perm,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                float* zeros, int32_t* g_idx, float* losses, void* ws,
+                                size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * gptq_pack — packing of low-bit codes into integer words (gptq-for-llama article,
+ * ainews.cool, "工程细节": four 4-bit codes per 16-bit integer).  Each row's codes
+ * form a little-endian, LSB-first bitstream of `bits`-bit fields:
+ *     code c occupies bits [c*bits, (c+1)*bits) of the row's stream,
+ * stored as rows x ceil(cols*bits/32) uint32 words; trailing bits are zero.  Codes
+ * are masked to `bits` bits.  bits in {2, 3, 4, 8}.  Errors: INVALID_ARG.
+ */
+gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits,
+                      uint32_t* packed, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* gptq_status_string(int status);
+
+/* Number of kernels this library has launched in the process (diagnostics). */
+uint64_t gptq_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPTQ_H_ */

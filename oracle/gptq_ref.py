@@ -248,7 +248,7 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bool,
             if h != z[r]:
                 if h in cand:
                     z[r] = np.float32(h)
-                    forced["zeros"].append((int(r), int(col_group)))
+                    forced["zeros"].append((int(r), int(col_group), float(_tie_distance(tz[r]))))
                 else:
                     forced["bad_hint"].append(("zero", int(r), int(col_group)))
         return z
@@ -281,7 +281,7 @@ def sweep(Wp: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bool,
                         if h in cand:
                             c[r] = h
                             Qq[r] = float(s[r]) * (h - float(z[r]))
-                            forced["codes"].append((int(r), int(q)))
+                            forced["codes"].append((int(r), int(q), float(_tie_distance(t[r]))))
                         else:
                             forced["bad_hint"].append(("code", int(r), int(q)))
             d = U[q, q]

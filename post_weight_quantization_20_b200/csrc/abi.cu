@@ -1,0 +1,125 @@
+// The C ABI of libgptq (include/gptq.h): argument validation and dispatch.
+// Every host-checkable error is reported before anything is launched.
+#include <atomic>
+#include <climits>
+#include <cmath>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gptq {
+static std::atomic<uint64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace gptq
+
+using namespace gptq;
+
+static bool valid_dtype(int dt) { return dt == GPTQ_F32 || dt == GPTQ_F16 || dt == GPTQ_BF16; }
+
+static gptq_status check_cfg(const gptq_config* cfg) {
+  if (!cfg) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->bits != 2 && cfg->bits != 3 && cfg->bits != 4 && cfg->bits != 8)
+    return GPTQ_ERR_INVALID_ARG;
+  if (cfg->sym != 0 && cfg->sym != 1) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->act_order < GPTQ_ORDER_NATURAL || cfg->act_order > GPTQ_ORDER_GIVEN)
+    return GPTQ_ERR_INVALID_ARG;
+  if (!(cfg->damp >= 0.f) || !std::isfinite(cfg->damp)) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->block_size < 1) return GPTQ_ERR_INVALID_ARG;
+  if (cfg->group_size < -1) return GPTQ_ERR_INVALID_ARG;
+  return GPTQ_OK;
+}
+
+static gptq_status check_group(const gptq_config* cfg) {
+  const int g = cfg->group_size;
+  if (g <= 0) return GPTQ_OK;
+  if (128 % g != 0) return GPTQ_ERR_UNSUPPORTED;
+  const int B = cfg->block_size;
+  if (g % B != 0 && B % g != 0) return GPTQ_ERR_UNSUPPORTED;
+  return GPTQ_OK;
+}
+
+static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+extern "C" {
+
+size_t gptq_workspace_size(int op, int64_t rows, int64_t cols, const gptq_config* cfg) {
+  if (cols <= 0 || cols > INT_MAX / 2 || rows < 0 || rows > INT_MAX) return 0;
+  if (check_cfg(cfg) != GPTQ_OK) return 0;
+  if (op == GPTQ_OP_PREPARE) return prepare_ws_bytes(cols);
+  if (op == GPTQ_OP_QUANTIZE) return quantize_ws_bytes(rows, cols, *cfg);
+  return 0;
+}
+
+gptq_status gptq_hessian_accumulate(float* H, int64_t* n_seen, const void* X, int xdtype,
+                                    int64_t m_tokens, int64_t cols, int64_t ldx,
+                                    int32_t* dev_status, void* stream) {
+  if (!H || !n_seen || cols <= 0 || cols > INT_MAX / 2 || m_tokens < 0 || *n_seen < 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (!valid_dtype(xdtype) || ldx < cols) return GPTQ_ERR_INVALID_ARG;
+  if (m_tokens == 0) return GPTQ_OK;
+  if (!X) return GPTQ_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  const int64_t n = *n_seen;
+  const double tot = double(n) + double(m_tokens);
+  GPTQ_TRY(hessian_prescale(st, H, int(cols), double(n) / tot, n == 0));
+  const float beta = float(2.0 / tot);
+  gptq_status s = hessian_syrk_tc(st, H, X, xdtype, m_tokens, int(cols), ldx, beta, dev_status);
+  if (s == GPTQ_ERR_UNSUPPORTED)
+    s = hessian_syrk_simt(st, H, X, xdtype, m_tokens, int(cols), ldx, beta);
+  if (s != GPTQ_OK) return s;
+  *n_seen = n + m_tokens;
+  return GPTQ_OK;
+}
+
+gptq_status gptq_prepare(const float* H, int64_t cols, const gptq_config* cfg, float* U,
+                         int32_t* perm, void* ws, size_t ws_bytes, int32_t* dev_status,
+                         void* stream) {
+  if (!H || !U || !perm || cols <= 0 || cols > INT_MAX / 2) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_TRY(check_cfg(cfg));
+  if (!ws || !aligned256(ws)) return GPTQ_ERR_INVALID_ARG;
+  if (ws_bytes < prepare_ws_bytes(cols)) return GPTQ_ERR_WORKSPACE;
+  return prepare_run(as_stream(stream), H, int(cols), *cfg, U, perm, ws, dev_status);
+}
+
+gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t cols,
+                                int64_t ldw, const float* U, const int32_t* perm,
+                                const gptq_config* cfg, uint8_t* codes, float* scales,
+                                float* zeros, int32_t* g_idx, float* losses, void* ws,
+                                size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (cols <= 0 || cols > INT_MAX / 2 || rows < 0 || rows > INT_MAX) return GPTQ_ERR_INVALID_ARG;
+  if (!U || !perm || !g_idx || !losses) return GPTQ_ERR_INVALID_ARG;
+  if (rows > 0 && (!W || !codes || !scales || !zeros)) return GPTQ_ERR_INVALID_ARG;
+  if (!valid_dtype(wdtype) || ldw < cols) return GPTQ_ERR_INVALID_ARG;
+  GPTQ_TRY(check_cfg(cfg));
+  GPTQ_TRY(check_group(cfg));
+  if (!ws || !aligned256(ws)) return GPTQ_ERR_INVALID_ARG;
+  if (ws_bytes < quantize_ws_bytes(rows, cols, *cfg)) return GPTQ_ERR_WORKSPACE;
+  return quantize_run(as_stream(stream), W, wdtype, int(rows), int(cols), ldw, U, perm, *cfg,
+                      codes, scales, zeros, g_idx, losses, ws, dev_status);
+}
+
+gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits,
+                      uint32_t* packed, void* stream) {
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return GPTQ_ERR_INVALID_ARG;
+  if (rows > 0 && cols > 0 && (!codes || !packed)) return GPTQ_ERR_INVALID_ARG;
+  return pack_run(as_stream(stream), codes, rows, cols, bits, packed);
+}
+
+const char* gptq_status_string(int status) {
+  switch (status) {
+    case GPTQ_OK: return "GPTQ_OK";
+    case GPTQ_ERR_INVALID_ARG: return "GPTQ_ERR_INVALID_ARG";
+    case GPTQ_ERR_UNSUPPORTED: return "GPTQ_ERR_UNSUPPORTED";
+    case GPTQ_ERR_WORKSPACE: return "GPTQ_ERR_WORKSPACE";
+    case GPTQ_ERR_NOT_PD: return "GPTQ_ERR_NOT_PD";
+    case GPTQ_ERR_NONFINITE: return "GPTQ_ERR_NONFINITE";
+    case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT";
+    case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA";
+    default: return "GPTQ_ERR_<combined>";
+  }
+}
+
+uint64_t gptq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

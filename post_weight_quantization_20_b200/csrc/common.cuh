@@ -1,0 +1,49 @@
+// Shared helpers of libgptq: status handling, launch accounting, element loads.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gptq.h"
+
+namespace gptq {
+
+void note_launch();  // counts every kernel launch issued by the library
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+__device__ __forceinline__ void raise_status(int32_t* st, int bits) {
+  if (st) atomicOr(st, bits);
+}
+
+__device__ __forceinline__ float load_f32(const void* p, int dt, int64_t idx) {
+  if (dt == GPTQ_F32) return static_cast<const float*>(p)[idx];
+  if (dt == GPTQ_F16) return __half2float(static_cast<const __half*>(p)[idx]);
+  return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[idx]);
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory (idempotent).
+template <typename K>
+inline cudaError_t allow_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+}  // namespace gptq
+
+// Launch a kernel, count it, and turn a launch error into GPTQ_ERR_CUDA.
+#define GPTQ_LAUNCH(kernel, grid, block, smem, stream, ...)                 \
+  do {                                                                      \
+    kernel<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);             \
+    ::gptq::note_launch();                                                  \
+    if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;           \
+  } while (0)
+
+#define GPTQ_TRY(expr)                          \
+  do {                                          \
+    gptq_status s_ = (expr);                    \
+    if (s_ != GPTQ_OK) return s_;               \
+  } while (0)

@@ -1,0 +1,31 @@
+// Internal host-side entry points shared between the library's translation units.
+#pragma once
+#include "common.cuh"
+
+namespace gptq {
+
+// hessian.cu
+gptq_status hessian_prescale(cudaStream_t st, float* H, int C, double alpha, bool overwrite);
+gptq_status hessian_syrk_simt(cudaStream_t st, float* H, const void* X, int dt, int64_t m, int C,
+                              int64_t ldx, float beta);
+// hessian_tc.cu: returns GPTQ_ERR_UNSUPPORTED when the tensor-core path does not apply.
+gptq_status hessian_syrk_tc(cudaStream_t st, float* H, const void* X, int dt, int64_t m, int C,
+                            int64_t ldx, float beta, int32_t* status);
+
+// prepare.cu
+size_t prepare_ws_bytes(int64_t C);
+gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_config& cfg, float* U,
+                        int32_t* perm, void* ws, int32_t* status);
+
+// sweep.cu
+size_t quantize_ws_bytes(int64_t R, int64_t C, const gptq_config& cfg);
+gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, int64_t ldw,
+                         const float* U, const int32_t* perm, const gptq_config& cfg,
+                         uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
+                         float* losses, void* ws, int32_t* status);
+
+// pack.cu
+gptq_status pack_run(cudaStream_t st, const uint8_t* codes, int64_t R, int64_t C, int bits,
+                     uint32_t* packed);
+
+}  // namespace gptq

@@ -1,0 +1,280 @@
+// The column sweep, GPTQ量化算法深度解析 §2.2 (OBS compensation), §2.4 (fixed order,
+// lazy batch updates), §3.1 step 3-4.
+//
+// Data layout in HBM (workspace):
+//   Wk    rows x C fp32   working copy of W in sweep order (columns gathered by perm)
+//   Err   rows x 128 fp32 scaled errors (w - Q)/U[q][q] of the current panel
+//   cp    rows x C u8     codes in sweep order
+//   lpart tiles x C fp32  per-row-tile partial column losses (summed in finalize)
+//
+// Rows are independent once U is known, so the in-panel sweep runs one row per
+// SW_TPR threads: each thread keeps SW_CPT panel columns in registers, the
+// column being quantized is broadcast with a warp shuffle, and every thread of
+// the row applies the rank-1 compensation to its own columns using the panel's
+// U block held in shared memory.  Group grids are warp-shuffle min/max
+// reductions over the row's g columns.  The lazy trailing update
+// W[:, end:] -= Err * U[panel, end:] is a separate GEMM.
+#include <algorithm>
+
+#include "common.cuh"
+#include "gemm_f32.cuh"
+#include "kernels.h"
+
+namespace gptq {
+
+constexpr int SW_B = 128;                 // panel width (columns)
+constexpr int SW_TPR = 4;                 // threads per row
+constexpr int SW_CPT = SW_B / SW_TPR;     // panel columns owned by one thread
+constexpr int SW_ROWS = 32;               // rows per CTA
+constexpr int SW_THREADS = SW_ROWS * SW_TPR;
+constexpr int SW_LDU = SW_B + 4 * SW_TPR; // skewed U row: column c at c + 4*(c / SW_CPT)
+constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_B * (SW_THREADS / 32)) * 4;
+
+struct QuantLayout {
+  float* Wk;
+  float* Err;
+  uint8_t* cp;
+  float* lpart;
+  int tiles;
+};
+
+static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
+  QuantLayout L{};
+  L.tiles = int((R + SW_ROWS - 1) / SW_ROWS);
+  char* p = static_cast<char*>(ws);
+  L.Wk = reinterpret_cast<float*>(p);   p += align256(size_t(R) * C * 4);
+  L.Err = reinterpret_cast<float*>(p);  p += align256(size_t(R) * SW_B * 4);
+  L.cp = reinterpret_cast<uint8_t*>(p); p += align256(size_t(R) * C);
+  L.lpart = reinterpret_cast<float*>(p);
+  return L;
+}
+
+size_t quantize_ws_bytes(int64_t R, int64_t C, const gptq_config&) {
+  const int64_t tiles = (R + SW_ROWS - 1) / SW_ROWS;
+  return align256(size_t(R) * C * 4) + align256(size_t(R) * SW_B * 4) + align256(size_t(R) * C) +
+         align256(size_t(tiles) * C * 4) + 256;
+}
+
+// Grid of a set of values with range [lo, hi] (lo <= 0 <= hi), all in IEEE fp32.
+__device__ __forceinline__ void grid_params(float lo, float hi, float maxq, int sym, float& s,
+                                            float& z) {
+  if (sym) {
+    float m = fmaxf(-lo, hi);
+    if (m == 0.f) m = 1.f;
+    s = __fdiv_rn(__fsub_rn(m, -m), maxq);
+    z = (maxq + 1.f) * 0.5f;
+  } else {
+    if (lo == 0.f && hi == 0.f) { lo = -1.f; hi = 1.f; }
+    s = __fdiv_rn(__fsub_rn(hi, lo), maxq);
+    z = rintf(__fdiv_rn(-lo, s));
+  }
+}
+
+// Wk[r][j] = W[r][perm[j]] as fp32.
+__global__ void k_load_w(const void* W, int dt, int R, int C, int64_t ldw, const int32_t* perm,
+                         float* Wk) {
+  const int64_t total = int64_t(R) * C;
+  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int r = int(idx / C), j = int(idx % C);
+    int p = perm[j];
+    p = min(max(p, 0), C - 1);
+    Wk[idx] = load_f32(W, dt, int64_t(r) * ldw + p);
+  }
+}
+
+// One grid per row from the uncompensated row (group_size 0): one warp per row.
+__global__ void k_row_grid(const float* Wk, int R, int C, int bits, int sym, float* scales,
+                           float* zeros) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= R) return;
+  const float* row = Wk + int64_t(warp) * C;
+  float lo = 0.f, hi = 0.f;
+  for (int j = lane; j < C; j += 32) {
+    lo = fminf(lo, row[j]);
+    hi = fmaxf(hi, row[j]);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    float s, z;
+    grid_params(lo, hi, float((1 << bits) - 1), sym, s, z);
+    scales[warp] = s;
+    zeros[warp] = z;
+  }
+}
+
+// In-panel sweep of columns [i0, i0 + nb) for SW_ROWS rows per CTA.
+__global__ void __launch_bounds__(SW_THREADS)
+k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits, int g, int sym,
+              float* scales, float* zeros, int G, uint8_t* cp, float* Err, float* lpart) {
+  extern __shared__ float sm[];
+  float* Us = sm;                       // SW_B x SW_LDU
+  float* dinv = Us + SW_B * SW_LDU;     // SW_B
+  float* red = dinv + SW_B;             // warps x SW_B
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int t = tid % SW_TPR;
+  const int r = blockIdx.x * SW_ROWS + tid / SW_TPR;
+  const bool rv = r < R;
+  for (int e = tid; e < SW_B * SW_B; e += SW_THREADS) {
+    const int a = e / SW_B, b = e % SW_B;
+    const float v = (a < nb && b < nb) ? U[int64_t(i0 + a) * C + i0 + b] : 0.f;
+    Us[a * SW_LDU + b + 4 * (b / SW_CPT)] = v;
+  }
+  if (tid < SW_B) dinv[tid] = tid < nb ? 1.f / U[int64_t(i0 + tid) * C + i0 + tid] : 0.f;
+  float w[SW_CPT];
+  const float* wrow = Wk + int64_t(rv ? r : 0) * C + i0 + t * SW_CPT;
+#pragma unroll
+  for (int jj = 0; jj < SW_CPT; ++jj) w[jj] = (rv && t * SW_CPT + jj < nb) ? wrow[jj] : 0.f;
+  __syncthreads();
+
+  const float maxq = float((1 << bits) - 1);
+  float s = 1.f, z = 0.f;
+  if (g <= 0 && rv) { s = scales[r]; z = zeros[r]; }
+  float e[SW_CPT];
+  uint32_t cw[SW_CPT / 4];
+#pragma unroll
+  for (int jj = 0; jj < SW_CPT; ++jj) e[jj] = 0.f;
+#pragma unroll
+  for (int jj = 0; jj < SW_CPT / 4; ++jj) cw[jj] = 0u;
+
+  for (int c = 0; c < SW_TPR; ++c) {
+#pragma unroll
+    for (int qq = 0; qq < SW_CPT; ++qq) {
+      const int q = c * SW_CPT + qq;
+      if (q >= nb) break;
+      if (g > 0 && (q % g) == 0) {
+        float lo = 0.f, hi = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < SW_CPT; ++jj) {
+          const int col = t * SW_CPT + jj;
+          if (col >= q && col < q + g && col < nb) {
+            lo = fminf(lo, w[jj]);
+            hi = fmaxf(hi, w[jj]);
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < SW_TPR; o <<= 1) {
+          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+        }
+        grid_params(lo, hi, maxq, sym, s, z);
+        if (t == 0 && rv) {
+          const int gi = (i0 + q) / g;
+          scales[int64_t(r) * G + gi] = s;
+          zeros[int64_t(r) * G + gi] = z;
+        }
+      }
+      const float x = __shfl_sync(0xffffffffu, w[qq], (lane & ~(SW_TPR - 1)) | c);
+      const float code = fminf(fmaxf(rintf(__fdiv_rn(x, s)) + z, 0.f), maxq);
+      const float Q = s * (code - z);
+      const float err = (x - Q) * dinv[q];
+      if (t == c) {
+        e[qq] = err;
+        cw[qq >> 2] |= uint32_t(code) << (8 * (qq & 3));
+      }
+      const float* urow = Us + q * SW_LDU + t * (SW_CPT + 4);
+#pragma unroll
+      for (int jj = 0; jj < SW_CPT; jj += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(urow + jj);
+        w[jj + 0] = fmaf(-err, u.x, w[jj + 0]);
+        w[jj + 1] = fmaf(-err, u.y, w[jj + 1]);
+        w[jj + 2] = fmaf(-err, u.z, w[jj + 2]);
+        w[jj + 3] = fmaf(-err, u.w, w[jj + 3]);
+      }
+    }
+  }
+
+  // errors for the trailing update, codes, and partial column losses
+  if (rv) {
+    float* erow = Err + int64_t(r) * SW_B + t * SW_CPT;
+    uint8_t* crow = cp + int64_t(r) * C + i0 + t * SW_CPT;
+#pragma unroll
+    for (int jj = 0; jj < SW_CPT; ++jj) {
+      const int col = t * SW_CPT + jj;
+      erow[jj] = e[jj];
+      if (col < nb) crow[jj] = uint8_t((cw[jj >> 2] >> (8 * (jj & 3))) & 0xffu);
+    }
+  }
+#pragma unroll
+  for (int jj = 0; jj < SW_CPT; ++jj) {
+    float l = rv ? 0.5f * e[jj] * e[jj] : 0.f;
+    l += __shfl_xor_sync(0xffffffffu, l, 4);
+    l += __shfl_xor_sync(0xffffffffu, l, 8);
+    l += __shfl_xor_sync(0xffffffffu, l, 16);
+    if (lane < SW_TPR) red[warp * SW_B + t * SW_CPT + jj] = l;
+  }
+  __syncthreads();
+  if (tid < nb) {
+    float l = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < SW_THREADS / 32; ++wi) l += red[wi * SW_B + tid];
+    lpart[int64_t(blockIdx.x) * C + i0 + tid] = l;
+  }
+}
+
+// Original column order: codes[r][perm[j]] = cp[r][j]; losses[perm[j]] = sum over
+// row tiles; g_idx[perm[j]] = j / g.
+__global__ void k_scatter_codes(const uint8_t* cp, int R, int C, const int32_t* perm,
+                                uint8_t* codes) {
+  const int64_t total = int64_t(R) * C;
+  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int r = int(idx / C), j = int(idx % C);
+    int p = perm[j];
+    p = min(max(p, 0), C - 1);
+    codes[int64_t(r) * C + p] = cp[idx];
+  }
+}
+
+__global__ void k_finalize_cols(const float* lpart, int tiles, int C, const int32_t* perm, int g,
+                                float* losses, int32_t* g_idx) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= C) return;
+  float l = 0.f;
+  for (int t = 0; t < tiles; ++t) l += lpart[int64_t(t) * C + j];
+  int p = perm[j];
+  p = min(max(p, 0), C - 1);
+  losses[p] = l;
+  g_idx[p] = g > 0 ? j / g : 0;
+}
+
+static int grid_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 32)); }
+
+gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, int64_t ldw,
+                         const float* U, const int32_t* perm, const gptq_config& cfg,
+                         uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
+                         float* losses, void* ws, int32_t* status) {
+  (void)status;
+  QuantLayout L = quant_layout(ws, R, C);
+  const int g = cfg.group_size > 0 ? cfg.group_size : 0;
+  const int G = g ? (C + g - 1) / g : 1;
+  if (R == 0) {
+    GPTQ_LAUNCH(k_finalize_cols, (C + 255) / 256, 256, 0, st, L.lpart, 0, C, perm, g, losses, g_idx);
+    return GPTQ_OK;
+  }
+  if (allow_smem(k_sweep_panel, SW_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
+  GPTQ_LAUNCH(k_load_w, grid_for(int64_t(R) * C), 256, 0, st, W, wdt, R, C, ldw, perm, L.Wk);
+  if (!g) {
+    GPTQ_LAUNCH(k_row_grid, (R + 7) / 8, 256, 0, st, L.Wk, R, C, cfg.bits, cfg.sym, scales, zeros);
+  }
+  for (int i0 = 0; i0 < C; i0 += SW_B) {
+    const int nb = min(SW_B, C - i0);
+    GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
+                g, cfg.sym, scales, zeros, G, L.cp, L.Err, L.lpart);
+    const int e = i0 + nb;
+    if (e < C) {
+      // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]
+      GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Err, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
+                        1.f, L.Wk + e, C, 0));
+    }
+  }
+  GPTQ_LAUNCH(k_scatter_codes, grid_for(int64_t(R) * C), 256, 0, st, L.cp, R, C, perm, codes);
+  GPTQ_LAUNCH(k_finalize_cols, (C + 255) / 256, 256, 0, st, L.lpart, L.tiles, C, perm, g, losses,
+              g_idx);
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -1,0 +1,346 @@
+"""Python binding of libgptq.so (ctypes): argument marshalling only.
+
+Every function named ``gptq_*`` mirrors the C call of the same name in
+``include/gptq.h``; tensors are passed as device pointers and every step of the
+solver runs in the library's CUDA kernels.  There is no CPU fallback: if the
+library is missing or no CUDA device is present, the calls raise.
+
+``quantize_layer`` strings the four calls together for one linear layer
+(GPTQ量化算法深度解析 §3.1 steps 1-4) and allocates the outputs with PyTorch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "lib", "libgptq.so")
+
+GPTQ_OK = 0
+GPTQ_ERR_INVALID_ARG = 1
+GPTQ_ERR_UNSUPPORTED = 2
+GPTQ_ERR_WORKSPACE = 4
+GPTQ_ERR_NOT_PD = 8
+GPTQ_ERR_NONFINITE = 16
+GPTQ_ERR_TIMEOUT = 32
+GPTQ_ERR_CUDA = 64
+
+GPTQ_F32, GPTQ_F16, GPTQ_BF16 = 0, 1, 2
+GPTQ_ORDER_NATURAL, GPTQ_ORDER_DESC_DIAG, GPTQ_ORDER_GIVEN = 0, 1, 2
+GPTQ_OP_PREPARE, GPTQ_OP_QUANTIZE = 1, 2
+
+_DT = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF16}
+
+# every symbol include/gptq.h declares
+EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare",
+           "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count")
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {status_names(code)}")
+
+
+def status_names(code: int) -> str:
+    if code == 0:
+        return "GPTQ_OK"
+    names = ["INVALID_ARG", "UNSUPPORTED", "WORKSPACE", "NOT_PD", "NONFINITE", "TIMEOUT", "CUDA"]
+    return "|".join("GPTQ_ERR_" + n for i, n in enumerate(names) if code & (1 << i))
+
+
+class gptq_config(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int), ("group_size", ctypes.c_int), ("sym", ctypes.c_int),
+                ("act_order", ctypes.c_int), ("damp", ctypes.c_float),
+                ("block_size", ctypes.c_int)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgptq.so (once) and declare the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built; run `python -m post_weight_quantization_20_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    cfgp = ctypes.POINTER(gptq_config)
+    lib.gptq_workspace_size.argtypes = [i32, i64, i64, cfgp]
+    lib.gptq_workspace_size.restype = sz
+    lib.gptq_hessian_accumulate.argtypes = [vp, ctypes.POINTER(i64), vp, i32, i64, i64, i64, vp, vp]
+    lib.gptq_hessian_accumulate.restype = i32
+    lib.gptq_prepare.argtypes = [vp, i64, cfgp, vp, vp, vp, sz, vp, vp]
+    lib.gptq_prepare.restype = i32
+    lib.gptq_quantize_layer.argtypes = [vp, i32, i64, i64, i64, vp, vp, cfgp, vp, vp, vp, vp, vp,
+                                        vp, sz, vp, vp]
+    lib.gptq_quantize_layer.restype = i32
+    lib.gptq_pack.argtypes = [vp, i64, i64, i32, vp, vp]
+    lib.gptq_pack.restype = i32
+    lib.gptq_status_string.argtypes = [i32]
+    lib.gptq_status_string.restype = ctypes.c_char_p
+    lib.gptq_launch_count.argtypes = []
+    lib.gptq_launch_count.restype = ctypes.c_uint64
+    _lib = lib
+    return lib
+
+
+def make_config(bits=4, group_size=128, sym=False, act_order=False, damp=0.01, block_size=128):
+    order = act_order if isinstance(act_order, int) and not isinstance(act_order, bool) else \
+        (GPTQ_ORDER_DESC_DIAG if act_order else GPTQ_ORDER_NATURAL)
+    return gptq_config(int(bits), int(group_size), int(bool(sym)), int(order), float(damp),
+                       int(block_size))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(code: int, where: str):
+    if code != GPTQ_OK:
+        raise GPTQError(code, where)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libgptq takes device tensors")
+
+
+# --------------------------------------------------------------------------- the C calls
+def gptq_workspace_size(op: int, rows: int, cols: int, cfg: gptq_config) -> int:
+    return int(load_library().gptq_workspace_size(op, rows, cols, ctypes.byref(cfg)))
+
+
+def gptq_hessian_accumulate(H: torch.Tensor, n_seen: int, X: torch.Tensor, status=None,
+                            stream=None) -> int:
+    """H (C x C fp32), X (m x C, row stride X.stride(0)); returns the new token count."""
+    _need_cuda(H, X, status)
+    n = ctypes.c_int64(int(n_seen))
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be 2-D with unit column stride")
+    code = load_library().gptq_hessian_accumulate(
+        _ptr(H), ctypes.byref(n), _ptr(X), _DT[X.dtype], X.shape[0], X.shape[1], X.stride(0),
+        _ptr(status), _stream(stream))
+    _check(code, "gptq_hessian_accumulate")
+    return int(n.value)
+
+
+def gptq_prepare(H, cfg, U, perm, ws, status=None, stream=None) -> None:
+    _need_cuda(H, U, perm, ws, status)
+    code = load_library().gptq_prepare(_ptr(H), H.shape[0], ctypes.byref(cfg), _ptr(U),
+                                       _ptr(perm), _ptr(ws), ws.numel() * ws.element_size(),
+                                       _ptr(status), _stream(stream))
+    _check(code, "gptq_prepare")
+
+
+def gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws, status=None,
+                        stream=None) -> None:
+    _need_cuda(W, U, perm, codes, scales, zeros, g_idx, losses, ws, status)
+    if W.dim() != 2 or W.stride(1) != 1:
+        raise ValueError("W must be 2-D with unit column stride")
+    code = load_library().gptq_quantize_layer(
+        _ptr(W), _DT[W.dtype], W.shape[0], W.shape[1], W.stride(0), _ptr(U), _ptr(perm),
+        ctypes.byref(cfg), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(losses),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(status), _stream(stream))
+    _check(code, "gptq_quantize_layer")
+
+
+def gptq_pack(codes, bits, packed, stream=None) -> None:
+    _need_cuda(codes, packed)
+    code = load_library().gptq_pack(_ptr(codes), codes.shape[0], codes.shape[1], int(bits),
+                                    _ptr(packed), _stream(stream))
+    _check(code, "gptq_pack")
+
+
+def gptq_status_string(code: int) -> str:
+    return load_library().gptq_status_string(int(code)).decode()
+
+
+def gptq_launch_count() -> int:
+    return int(load_library().gptq_launch_count())
+
+
+# --------------------------------------------------------------------------- one layer
+def packed_words(cols: int, bits: int) -> int:
+    return (cols * bits + 31) // 32
+
+
+def n_groups(cols: int, group_size: int) -> int:
+    return (cols + group_size - 1) // group_size if group_size > 0 else 1
+
+
+def alloc_workspace(op: int, rows: int, cols: int, cfg: gptq_config, device) -> torch.Tensor:
+    nbytes = gptq_workspace_size(op, rows, cols, cfg)
+    if nbytes == 0:
+        raise GPTQError(GPTQ_ERR_INVALID_ARG, "gptq_workspace_size")
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+@dataclass
+class LayerResult:
+    codes: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    g_idx: torch.Tensor
+    losses: torch.Tensor
+    perm: torch.Tensor
+    packed: torch.Tensor
+    H: torch.Tensor
+    U: torch.Tensor
+    n_tokens: int
+
+
+def check_status(status: torch.Tensor, where: str = "device") -> None:
+    code = int(status.item())
+    if code:
+        raise GPTQError(code, where)
+
+
+def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | None = None,
+                   chunk_tokens: int | None = None, stream=None, check: bool = True) -> LayerResult:
+    """Quantize one linear layer.  W (rows x cols) and X (tokens x cols, or an
+    iterable of such chunks) are device tensors."""
+    dev = W.device
+    R, C = W.shape
+    H = torch.empty(C, C, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = 0
+    chunks = [X] if isinstance(X, torch.Tensor) else X
+    for Xc in chunks:
+        if chunk_tokens:
+            for t0 in range(0, Xc.shape[0], chunk_tokens):
+                n = gptq_hessian_accumulate(H, n, Xc[t0:t0 + chunk_tokens], status, stream)
+        else:
+            n = gptq_hessian_accumulate(H, n, Xc, status, stream)
+    U = torch.empty(C, C, dtype=torch.float32, device=dev)
+    if perm is None:
+        perm = torch.empty(C, dtype=torch.int32, device=dev)
+    ws = alloc_workspace(GPTQ_OP_PREPARE, R, C, cfg, dev)
+    gptq_prepare(H, cfg, U, perm, ws, status, stream)
+    del ws
+    G = n_groups(C, cfg.group_size)
+    codes = torch.empty(R, C, dtype=torch.uint8, device=dev)
+    scales = torch.empty(R, G, dtype=torch.float32, device=dev)
+    zeros = torch.empty(R, G, dtype=torch.float32, device=dev)
+    g_idx = torch.empty(C, dtype=torch.int32, device=dev)
+    losses = torch.empty(C, dtype=torch.float32, device=dev)
+    ws = alloc_workspace(GPTQ_OP_QUANTIZE, R, C, cfg, dev)
+    gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws, status, stream)
+    packed = torch.empty(R, packed_words(C, cfg.bits), dtype=torch.int32, device=dev)
+    gptq_pack(codes, cfg.bits, packed, stream)
+    if check:
+        check_status(status, "quantize_layer")
+    return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n)
+
+
+# --------------------------------------------------------------------------- host buffers
+@dataclass
+class HostResult:
+    """Quantized layer copied back to (pinned) host memory."""
+    packed: torch.Tensor
+    scales: torch.Tensor
+    zeros: torch.Tensor
+    g_idx: torch.Tensor
+    losses: torch.Tensor
+    perm: torch.Tensor
+    status: torch.Tensor
+
+    @property
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.packed, self.scales, self.zeros, self.g_idx, self.losses, self.perm,
+                    self.status))
+
+
+_copy_streams: dict = {}
+_pinned_cache: dict = {}
+
+
+def _side_stream(dev) -> torch.cuda.Stream:
+    key = torch.device(dev).index
+    if key not in _copy_streams:
+        _copy_streams[key] = torch.cuda.Stream(device=dev)
+    return _copy_streams[key]
+
+
+def _pinned(key, shape, dtype) -> torch.Tensor:
+    k = (key, tuple(shape), dtype)
+    if k not in _pinned_cache:
+        _pinned_cache[k] = torch.empty(shape, dtype=dtype, pin_memory=True)
+    return _pinned_cache[k]
+
+
+def quantize_layer_host(W_host: torch.Tensor, X_host: torch.Tensor, cfg: gptq_config, device=None,
+                        chunk_tokens: int = 32768, stream=None, tag: str = "") -> HostResult:
+    """Quantize one layer whose W and X live in pinned host memory.
+
+    X is uploaded in chunks on a side stream while the previous chunk is being
+    accumulated into H on the compute stream (two device staging buffers); the
+    packed codes, scales, zeros, g_idx, losses and perm are copied back into
+    pinned host tensors.  Asynchronous: synchronize the stream before reading
+    the result (result.status holds the device status word).
+    """
+    dev = torch.device(device) if device is not None else torch.device("cuda")
+    comp = stream if stream is not None else torch.cuda.current_stream(dev)
+    side = _side_stream(dev)
+    side.wait_stream(comp)          # earlier work on the staging memory is finished
+    R, C = W_host.shape
+    T = X_host.shape[0]
+    W = torch.empty((R, C), dtype=W_host.dtype, device=dev)
+    stage = [torch.empty((min(chunk_tokens, max(T, 1)), C), dtype=X_host.dtype, device=dev)
+             for _ in range(2)]
+    ready = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    with torch.cuda.stream(side):
+        W.copy_(W_host, non_blocking=True)
+    w_ready = torch.cuda.Event()
+    w_ready.record(side)
+    H = torch.empty(C, C, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    n = 0
+    for k, t0 in enumerate(range(0, T, chunk_tokens)):
+        m = min(chunk_tokens, T - t0)
+        b = k % 2
+        if k >= 2:
+            side.wait_event(done[b])
+        with torch.cuda.stream(side):
+            stage[b][:m].copy_(X_host[t0:t0 + m], non_blocking=True)
+        ready[b].record(side)
+        comp.wait_event(ready[b])
+        n = gptq_hessian_accumulate(H, n, stage[b][:m], status, comp)
+        done[b].record(comp)
+    comp.wait_event(w_ready)
+    U = torch.empty(C, C, dtype=torch.float32, device=dev)
+    perm = torch.empty(C, dtype=torch.int32, device=dev)
+    with torch.cuda.stream(comp):
+        wsp = alloc_workspace(GPTQ_OP_PREPARE, R, C, cfg, dev)
+        gptq_prepare(H, cfg, U, perm, wsp, status, comp)
+        Gn = n_groups(C, cfg.group_size)
+        codes = torch.empty(R, C, dtype=torch.uint8, device=dev)
+        scales = torch.empty(R, Gn, dtype=torch.float32, device=dev)
+        zeros = torch.empty(R, Gn, dtype=torch.float32, device=dev)
+        g_idx = torch.empty(C, dtype=torch.int32, device=dev)
+        losses = torch.empty(C, dtype=torch.float32, device=dev)
+        wsq = alloc_workspace(GPTQ_OP_QUANTIZE, R, C, cfg, dev)
+        gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, wsq, status, comp)
+        packed = torch.empty(R, packed_words(C, cfg.bits), dtype=torch.int32, device=dev)
+        gptq_pack(codes, cfg.bits, packed, comp)
+        host = HostResult(*(_pinned((tag, i), t.shape, t.dtype) for i, t in
+                            enumerate((packed, scales, zeros, g_idx, losses, perm, status))))
+        for dst, src in zip((host.packed, host.scales, host.zeros, host.g_idx, host.losses,
+                             host.perm, host.status),
+                            (packed, scales, zeros, g_idx, losses, perm, status)):
+            dst.copy_(src, non_blocking=True)
+    return host

@@ -1,0 +1,117 @@
+"""The C-ABI library: it loads, exports every symbol include/gptq.h declares, and
+rejects bad arguments on the host before launching anything.  No compute calls."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from post_weight_quantization_20_b200 import gptq as G
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gptq.h")
+
+no_gpu = pytest.mark.skipif(torch.cuda.is_available(),
+                            reason="passes fake device pointers; only run without a GPU")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = G.load_library()
+    names = declared_functions()
+    assert len(names) == 7, names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(G.EXPORTS) == names
+
+
+def test_status_strings():
+    assert G.gptq_status_string(0) == "GPTQ_OK"
+    assert G.gptq_status_string(G.GPTQ_ERR_NOT_PD) == "GPTQ_ERR_NOT_PD"
+    assert G.status_names(G.GPTQ_ERR_NOT_PD | G.GPTQ_ERR_NONFINITE) == "GPTQ_ERR_NOT_PD|GPTQ_ERR_NONFINITE"
+
+
+def test_workspace_sizes():
+    cfg = G.make_config(4, 128)
+    a = G.gptq_workspace_size(G.GPTQ_OP_PREPARE, 0, 768, cfg)
+    b = G.gptq_workspace_size(G.GPTQ_OP_PREPARE, 0, 3072, cfg)
+    assert a > 2 * 768 * 768 * 4 and b > a and a % 256 == 0
+    q = G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, 3072, 768, cfg)
+    assert q >= 3072 * 768 * 5
+    assert G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, 10, 0, cfg) == 0
+    assert G.gptq_workspace_size(99, 10, 10, cfg) == 0
+    bad = G.make_config(5, 128)
+    assert G.gptq_workspace_size(G.GPTQ_OP_PREPARE, 0, 10, bad) == 0
+
+
+def _raw(name, *args):
+    return getattr(G.load_library(), name)(*args)
+
+
+def test_pack_rejects_bad_bits_and_nulls():
+    assert _raw("gptq_pack", None, 4, 4, 5, None, None) == G.GPTQ_ERR_INVALID_ARG
+    assert _raw("gptq_pack", None, 4, 4, 4, None, None) == G.GPTQ_ERR_INVALID_ARG
+    assert _raw("gptq_pack", None, -1, 4, 4, None, None) == G.GPTQ_ERR_INVALID_ARG
+    # empty input is a valid no-op
+    assert _raw("gptq_pack", None, 0, 7, 4, None, None) == G.GPTQ_OK
+
+
+def test_hessian_rejects_bad_arguments():
+    n = ctypes.c_int64(0)
+    f = G.load_library().gptq_hessian_accumulate
+    assert f(None, ctypes.byref(n), None, 1, 10, 8, 8, None, None) == G.GPTQ_ERR_INVALID_ARG
+    neg = ctypes.c_int64(-3)
+    assert f(ctypes.c_void_p(256), ctypes.byref(neg), None, 1, 10, 8, 8, None, None) == G.GPTQ_ERR_INVALID_ARG
+    # m == 0 is a no-op that touches nothing
+    assert f(ctypes.c_void_p(256), ctypes.byref(n), None, 1, 0, 8, 8, None, None) == G.GPTQ_OK
+    assert n.value == 0
+
+
+@no_gpu
+def test_hessian_rejects_bad_dtype_and_stride():
+    n = ctypes.c_int64(0)
+    f = G.load_library().gptq_hessian_accumulate
+    fake = ctypes.c_void_p(4096)
+    assert f(fake, ctypes.byref(n), fake, 7, 10, 8, 8, None, None) == G.GPTQ_ERR_INVALID_ARG
+    assert f(fake, ctypes.byref(n), fake, 1, 10, 8, 4, None, None) == G.GPTQ_ERR_INVALID_ARG
+
+
+@no_gpu
+def test_prepare_and_quantize_validation():
+    lib = G.load_library()
+    fake = ctypes.c_void_p(4096)
+    cfg = G.make_config(4, 128)
+    ws_need = G.gptq_workspace_size(G.GPTQ_OP_PREPARE, 0, 64, cfg)
+    assert lib.gptq_prepare(fake, 64, ctypes.byref(cfg), fake, fake, fake, ws_need - 1, None,
+                            None) == G.GPTQ_ERR_WORKSPACE
+    assert lib.gptq_prepare(fake, 64, ctypes.byref(cfg), fake, fake, ctypes.c_void_p(4100),
+                            ws_need, None, None) == G.GPTQ_ERR_INVALID_ARG  # unaligned ws
+    assert lib.gptq_prepare(fake, 64, None, fake, fake, fake, ws_need, None,
+                            None) == G.GPTQ_ERR_INVALID_ARG
+    q = G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, 8, 64, cfg)
+    for g, B, want in [(96, 128, G.GPTQ_ERR_UNSUPPORTED), (256, 128, G.GPTQ_ERR_UNSUPPORTED),
+                       (64, 48, G.GPTQ_ERR_UNSUPPORTED)]:
+        c = G.make_config(4, g, block_size=B)
+        assert lib.gptq_quantize_layer(fake, 1, 8, 64, 64, fake, fake, ctypes.byref(c), fake, fake,
+                                       fake, fake, fake, fake, q, None, None) == want
+    c = G.make_config(4, 64)
+    assert lib.gptq_quantize_layer(fake, 1, 8, 64, 32, fake, fake, ctypes.byref(c), fake, fake,
+                                   fake, fake, fake, fake, q, None, None) == G.GPTQ_ERR_INVALID_ARG
+    assert lib.gptq_quantize_layer(fake, 1, 8, 64, 64, fake, fake, ctypes.byref(c), fake, fake,
+                                   fake, fake, fake, fake, q - 1, None, None) == G.GPTQ_ERR_WORKSPACE
+    bad = G.make_config(4, 64, damp=float("nan"))
+    assert lib.gptq_quantize_layer(fake, 1, 8, 64, 64, fake, fake, ctypes.byref(bad), fake, fake,
+                                   fake, fake, fake, fake, q, None, None) == G.GPTQ_ERR_INVALID_ARG
+
+
+def test_binding_refuses_host_tensors():
+    H = torch.zeros(4, 4)
+    X = torch.zeros(8, 4)
+    with pytest.raises(ValueError):
+        G.gptq_hessian_accumulate(H, 0, X)
