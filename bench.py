@@ -36,6 +36,11 @@ from post_weight_quantization_20_b200.workloads import WORKLOADS  # noqa: E402
 
 METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per Hessian launch from the ncu capture summarised in
+# profiles/hessian_tc_C3072_T65536.md (C = 3072, 65536 tokens: 686.1 MB + 130.3 MB),
+# scaled to the bench's 262144-token launch by the token count.  Set to None when
+# the kernel changes until it is captured again.
+HESSIAN_TRAFFIC = {"bytes_per_token_C3072": (686.134272e6 + 130.278912e6) / 65536}
 
 
 def load_peaks():
@@ -252,6 +257,10 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     achieved = hess_flop / (hess_ms * 1e-3) / 1e12 if hess_ms > 0 else None
     peak = float(peaks["bf16_tflops"])
+    traffic = None
+    if HESSIAN_TRAFFIC and any(C == 3072 for _, _, _, C in hess_ev):
+        toks = [m for _, _, m, C in hess_ev if C == 3072][0]
+        traffic = HESSIAN_TRAFFIC["bytes_per_token_C3072"] * toks
     out = {
         "metric": METRIC,
         "value": ms / args.steps / n_layers,
@@ -270,7 +279,9 @@ def run_ours(args, rank, world, local_rank):
                     "launches": n_hess},
         "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (achieved / peak) if achieved else None, "traffic": None,
+                     "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                     "traffic_scope": "bytes per C=3072 launch (the largest Hessian of the "
+                                      "workload), ncu capture at 65536 tokens scaled by tokens",
                      "peak_source": f"{peaks['source']} bf16 dense burst"},
         "e2e": {"value": e2e_ms / len(layers), "unit": "ms", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},

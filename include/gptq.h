@@ -172,6 +172,11 @@ const char* gptq_status_string(int status);
 /* Number of kernels this library has launched in the process (diagnostics). */
 uint64_t gptq_launch_count(void);
 
+/* Description of the most recent CUDA failure seen by the calling thread inside the
+ * library (the call that returned GPTQ_ERR_CUDA), or "" if none.  Static per-thread
+ * string, overwritten by the next failure. */
+const char* gptq_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,9 +7,16 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <cstdio>
+
 namespace gptq {
 static std::atomic<uint64_t> g_launches{0};
+static thread_local char g_last_error[256] = "";
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void note_error(cudaError_t e, const char* where) {
+  std::snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e),
+                cudaGetErrorString(e));
+}
 }  // namespace gptq
 
 using namespace gptq;
@@ -121,5 +128,7 @@ const char* gptq_status_string(int status) {
 }
 
 uint64_t gptq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* gptq_last_error(void) { return g_last_error; }
 
 }  // extern "C"

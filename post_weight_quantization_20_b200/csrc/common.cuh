@@ -11,6 +11,7 @@
 namespace gptq {
 
 void note_launch();  // counts every kernel launch issued by the library
+void note_error(cudaError_t e, const char* where);  // remembers the last CUDA failure
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -39,7 +40,20 @@ inline cudaError_t allow_smem(K kernel, int bytes) {
   do {                                                                      \
     kernel<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);             \
     ::gptq::note_launch();                                                  \
-    if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;           \
+    const cudaError_t e_ = cudaGetLastError();                              \
+    if (e_ != cudaSuccess) {                                                \
+      ::gptq::note_error(e_, #kernel);                                      \
+      return GPTQ_ERR_CUDA;                                                 \
+    }                                                                       \
+  } while (0)
+
+#define GPTQ_CUDA(call)                                                     \
+  do {                                                                      \
+    const cudaError_t e_ = (call);                                          \
+    if (e_ != cudaSuccess) {                                                \
+      ::gptq::note_error(e_, #call);                                        \
+      return GPTQ_ERR_CUDA;                                                 \
+    }                                                                       \
   } while (0)
 
 #define GPTQ_TRY(expr)                          \

@@ -1,10 +1,319 @@
-// Placeholder for the tcgen05 Hessian contraction (replaced by the tensor-core kernel).
-#include "common.cuh"
+// Hessian contraction on the 5th-generation tensor cores:
+//   H[i][j] += beta * sum_t X[t][i] X[t][j]      (upper-triangle tiles, fp16/bf16 in, fp32 acc)
+// for GPTQ量化算法深度解析 §3.1 step 1.
+//
+// Output tile 128 (i) x 256 (j); both operands are read straight from row-major
+// X by TMA as 64-token x 64-column boxes with 128-byte swizzle, which is the
+// MN-major layout tcgen05 consumes (no transpose pass over X).  Per CTA:
+//   warp 0      TMA producer (4-stage ring, 48 KB per stage)
+//   warp 1      TMEM allocator and MMA issuer (tcgen05.mma kind::f16, M=128 N=256 K=16)
+//   warps 2-9   epilogue: two warps per TMEM lane quadrant, 128 columns each
+//
+// Precision: the tensor core's fp32 accumulation does not round to nearest, so
+// a long accumulation chain inside TMEM drifts (about 1e-4 relative over 20k
+// tokens).  The MMA therefore accumulates SEG token steps (256 tokens) into one
+// of two TMEM buffers, and the epilogue adds each segment into a register
+// accumulator with ordinary round-to-nearest fp32 adds while the MMA fills the
+// other buffer.  At the end of a work item the registers are added into H with
+// vector red.global.add.
+//
+// Work items are (tile, token split) pairs handed out round-robin to a
+// persistent grid of one CTA per SM; items in flight together share token
+// ranges, so X is re-read from L2 rather than HBM.  H's upper triangle has been
+// scaled by the running-mean factor beforehand, so every item adds its sum.
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace gptq {
-gptq_status hessian_syrk_tc(cudaStream_t, float*, const void*, int, int64_t, int, int64_t, float,
-                            int32_t*) {
-  return GPTQ_ERR_UNSUPPORTED;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;   // tile and tokens per stage
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_BYTES = BN * BK * 2;         // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int BOX_BYTES = 64 * BK * 2;       // one 64-column x 64-token box, 8 KB
+constexpr int THREADS = 320;                 // 2 control warps + 8 epilogue warps
+constexpr int SEG = 4;                       // token steps (of 64) per TMEM segment
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+
+struct Sched {
+  int C, T, S, kt, ntj, vec;
+};
+
+// t-th upper tile: j-tile jt holds i-tiles a = 0 .. min(nti, 2 jt + 2) - 1.
+__device__ __forceinline__ void tile_coords(const Sched& s, int t, int& i0, int& j0) {
+  const int nti = (s.C + BM - 1) / BM;
+  int jt = 0;
+  for (; jt < s.ntj; ++jt) {
+    const int cnt = min(nti, 2 * jt + 2);
+    if (t < cnt) break;
+    t -= cnt;
+  }
+  i0 = t * BM;
+  j0 = jt * BN;
 }
+
+__device__ __forceinline__ void item_range(const Sched& s, int w, int& t, int& k0, int& k1) {
+  const int sp = w / s.T;
+  t = w % s.T;
+  k0 = int((int64_t(s.kt) * sp) / s.S);
+  k1 = int((int64_t(s.kt) * (sp + 1)) / s.S);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, float beta,
+               uint32_t idesc, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_items = s.S * s.T;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      tc::mbar_init(full + i, 1);
+      tc::mbar_init(empty + i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(acc_full + i, 1);
+      tc::mbar_init(acc_empty + i, 8);
+    }
+    *abort_flag = 0;
+    tc::fence_barrier_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(tmem_slot, TMEM_COLS);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        int t, k0, k1, i0, j0;
+        item_range(s, w, t, k0, k1);
+        tile_coords(s, t, i0, j0);
+        for (int k = k0; k < k1; ++k) {
+          if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* a = smem + stage * STAGE_BYTES;
+          uint8_t* b = a + A_BYTES;
+          tc::mbar_expect_tx(full + stage, STAGE_BYTES);
+          const int y = k * BK;
+#pragma unroll
+          for (int q = 0; q < BM / 64; ++q) tc::tma_load_2d(a + q * BOX_BYTES, &xmap, i0 + 64 * q, y, full + stage);
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q) tc::tma_load_2d(b + q * BOX_BYTES, &xmap, j0 + 64 * q, y, full + stage);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        int t, k0, k1;
+        item_range(s, w, t, k0, k1);
+        for (int ks = k0; ks < k1 && ok; ks += SEG) {
+          const int ke = min(ks + SEG, k1);
+          if (!tc::mbar_wait(acc_empty + acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t d = tmem_base + uint32_t(acc * BN);
+          for (int k = ks; k < ke; ++k) {
+            if (!tc::mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint8_t* a = smem + stage * STAGE_BYTES;
+            const uint8_t* b = a + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // 16 tokens = 16 rows of 128 B inside each swizzled box
+              const uint64_t ad = tc::smem_desc_sw128(a + kk * 2048, BOX_BYTES, 1024);
+              const uint64_t bd = tc::smem_desc_sw128(b + kk * 2048, BOX_BYTES, 1024);
+              tc::mma_f16(d, ad, bd, idesc, (k > ks || kk > 0) ? 1u : 0u);
+            }
+            tc::mma_commit(empty + stage);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
+          if (!ok) break;
+          tc::mma_commit(acc_full + acc);
+          if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        }
+      }
+    }
+  } else {
+    // epilogue warps 2..9: TMEM lanes 32*(warp % 4) .. +31, columns 128*half .. +127
+    const int lane_base = (warp & 3) * 32;
+    const int half = (warp - 2) >> 2;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    const bool vec = s.vec != 0;
+    bool ok = true;
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      int t, k0, k1, i0, j0;
+      item_range(s, w, t, k0, k1);
+      tile_coords(s, t, i0, j0);
+      float r[128];
+#pragma unroll
+      for (int q = 0; q < 128; ++q) r[q] = 0.f;
+      for (int ks = k0; ks < k1; ks += SEG) {
+        if (!tc::mbar_wait(acc_full + acc, acc_phase, abort_flag)) { ok = false; break; }
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[16];
+          tc::tmem_ld_32x16(tmem_base + (uint32_t(lane_base) << 16) +
+                                uint32_t(acc * BN + half * 128 + c * 16), v);
+          tc::tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) r[c * 16 + q] += __uint_as_float(v[q]);
+        }
+        tc::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(acc_empty + acc);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok) break;
+      const int gi = i0 + lane_base + lane;
+      if (gi < s.C) {
+        float* hrow = H + int64_t(gi) * s.C;
+        const int jb = j0 + half * 128;
+#pragma unroll
+        for (int q = 0; q < 128; q += 4) {
+          const int gj = jb + q;
+          const float x0 = beta * r[q], x1 = beta * r[q + 1];
+          const float x2 = beta * r[q + 2], x3 = beta * r[q + 3];
+          if (vec && gj >= gi && gj + 3 < s.C) {
+            tc::red_add_v4(hrow + gj, x0, x1, x2, x3);
+          } else {
+            if (gj >= gi && gj < s.C) atomicAdd(hrow + gj, x0);
+            if (gj + 1 >= gi && gj + 1 < s.C) atomicAdd(hrow + gj + 1, x1);
+            if (gj + 2 >= gi && gj + 2 < s.C) atomicAdd(hrow + gj + 2, x2);
+            if (gj + 3 >= gi && gj + 3 < s.C) atomicAdd(hrow + gj + 3, x3);
+          }
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) raise_status(status, GPTQ_ERR_TIMEOUT);
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+static bool tc_supported_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  return major == 10 && minor == 0;
+}
+
+// Token splits per tile: the fewest that keep the last wave of the persistent
+// grid at least 95% full, and that keep every work item at or below 16384
+// token steps (a few ms) so no wait in the kernel comes near its limit.
+static int choose_splits(int T, int P, int kt) {
+  const int smin = std::max(1, (kt + 16383) / 16384);
+  int best = smin;
+  for (int S = smin; S <= smin + 64; ++S) {
+    if (S > kt) break;
+    const double items = double(S) * T;
+    const double waves = items / P;
+    const double eff = waves / std::ceil(waves);
+    best = S;
+    if (eff >= 0.95) break;
+  }
+  return best;
+}
+
+gptq_status hessian_syrk_tc(cudaStream_t st, float* H, const void* X, int dt, int64_t m, int C,
+                            int64_t ldx, float beta, int32_t* status) {
+  if (dt != GPTQ_F16 && dt != GPTQ_BF16) return GPTQ_ERR_UNSUPPORTED;
+  if ((ldx % 8) != 0 || (reinterpret_cast<uintptr_t>(X) & 15) != 0) return GPTQ_ERR_UNSUPPORTED;
+  if (m > (int64_t(1) << 31) - BK || !tc_supported_device()) return GPTQ_ERR_UNSUPPORTED;
+  EncodeTiledFn enc = encode_tiled_fn();
+  const int P = sm_count();
+  if (!enc || P <= 0) return GPTQ_ERR_UNSUPPORTED;
+
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(C), cuuint64_t(m)};
+  const cuuint64_t strides[1] = {cuuint64_t(ldx) * 2};
+  const cuuint32_t box[2] = {64, BK};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType ty =
+      dt == GPTQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (enc(&map, ty, 2, const_cast<void*>(X), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return GPTQ_ERR_UNSUPPORTED;
+
+  Sched s;
+  s.C = C;
+  s.ntj = (C + BN - 1) / BN;
+  const int nti = (C + BM - 1) / BM;
+  s.T = 0;
+  for (int jt = 0; jt < s.ntj; ++jt) s.T += std::min(nti, 2 * jt + 2);
+  s.kt = int((m + BK - 1) / BK);
+  s.S = choose_splits(s.T, P, s.kt);
+  s.vec = ((C & 3) == 0 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) ? 1 : 0;
+  const int items = s.S * s.T;
+  const int grid = std::min(P, items);
+
+  // idesc: D f32, A/B f16 or bf16, both MN-major, N = 256, M = 128
+  const uint32_t fmt = dt == GPTQ_F16 ? 0u : 1u;
+  const uint32_t idesc = (1u << 4) | (fmt << 7) | (fmt << 10) | (1u << 15) | (1u << 16) |
+                         (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+  GPTQ_CUDA(allow_smem(k_hess_syrk_tc, SMEM_BYTES));
+  GPTQ_LAUNCH(k_hess_syrk_tc, grid, THREADS, SMEM_BYTES, st, map, H, s, beta, idesc, status);
+  return GPTQ_OK;
+}
+
 }  // namespace gptq

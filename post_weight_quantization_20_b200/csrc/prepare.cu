@@ -210,7 +210,7 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
     GPTQ_LAUNCH(k_iota, pb, 256, 0, st, perm, C);
     GPTQ_LAUNCH(k_rank_perm, pb, 256, 0, st, L.diag, C, perm);
   } else {
-    if (cudaMemsetAsync(L.cnt, 0, size_t(C) * 4, st) != cudaSuccess) return GPTQ_ERR_CUDA;
+    GPTQ_CUDA(cudaMemsetAsync(L.cnt, 0, size_t(C) * 4, st));
     GPTQ_LAUNCH(k_perm_count, pb, 256, 0, st, perm, C, L.cnt, status);
     GPTQ_LAUNCH(k_perm_check, pb, 256, 0, st, L.cnt, C, status);
   }

@@ -255,7 +255,7 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
     GPTQ_LAUNCH(k_finalize_cols, (C + 255) / 256, 256, 0, st, L.lpart, 0, C, perm, g, losses, g_idx);
     return GPTQ_OK;
   }
-  if (allow_smem(k_sweep_panel, SW_SMEM) != cudaSuccess) return GPTQ_ERR_CUDA;
+  GPTQ_CUDA(allow_smem(k_sweep_panel, SW_SMEM));
   GPTQ_LAUNCH(k_load_w, grid_for(int64_t(R) * C), 256, 0, st, W, wdt, R, C, ldw, perm, L.Wk);
   if (!g) {
     GPTQ_LAUNCH(k_row_grid, (R + 7) / 8, 256, 0, st, L.Wk, R, C, cfg.bits, cfg.sym, scales, zeros);

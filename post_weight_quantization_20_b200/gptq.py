@@ -35,7 +35,8 @@ _DT = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF
 
 # every symbol include/gptq.h declares
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare",
-           "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count")
+           "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count",
+           "gptq_last_error")
 
 
 class GPTQError(RuntimeError):
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_status_string.restype = ctypes.c_char_p
     lib.gptq_launch_count.argtypes = []
     lib.gptq_launch_count.restype = ctypes.c_uint64
+    lib.gptq_last_error.argtypes = []
+    lib.gptq_last_error.restype = ctypes.c_char_p
     _lib = lib
     return lib
 
@@ -108,6 +111,8 @@ def _stream(stream):
 
 def _check(code: int, where: str):
     if code != GPTQ_OK:
+        if code == GPTQ_ERR_CUDA:
+            where = f"{where} [{gptq_last_error()}]"
         raise GPTQError(code, where)
 
 
@@ -169,6 +174,10 @@ def gptq_status_string(code: int) -> str:
 
 def gptq_launch_count() -> int:
     return int(load_library().gptq_launch_count())
+
+
+def gptq_last_error() -> str:
+    return load_library().gptq_last_error().decode()
 
 
 # --------------------------------------------------------------------------- one layer

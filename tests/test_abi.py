@@ -25,10 +25,14 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = G.load_library()
     names = declared_functions()
-    assert len(names) == 7, names
+    assert len(names) == 8, names
     for n in names:
         assert hasattr(lib, n), n
     assert sorted(G.EXPORTS) == names
+
+
+def test_last_error_starts_empty():
+    assert G.gptq_last_error() == ""
 
 
 def test_status_strings():

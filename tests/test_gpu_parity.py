@@ -25,11 +25,6 @@ TAU = 2e-3          # grid steps: fp32 state vs fp64 state (see design notes)
 DEV = "cuda"
 
 
-def _dev(a, dtype=None):
-    t = torch.from_numpy(np.ascontiguousarray(a))
-    if dtype is not None:
-        t = t.view(dtype) if t.dtype == torch.int16 or a.dtype == np.uint16 else t.to(dtype)
-    return t.to(DEV)
 
 
 def to_device(arr, sdtype):
@@ -256,3 +251,32 @@ def test_act_order_perm_from_device_hessian():
     # descending in the oracle's diagonal, up to fp32 accumulation error at near-ties
     dp = d[perm]
     assert np.all(dp[:-1] >= dp[1:] - 1e-5 * np.abs(dp[1:]))
+
+
+# --------------------------------------------------------------------------- full-size sampled checks
+@pytest.mark.parametrize("layer", ["fc1", "fc2"])
+def test_hessian_full_size_sampled_entries(layer):
+    """Bench workload shapes (262144 calibration tokens, as launched by bench.py):
+    sampled entries H[i][j] against the oracle evaluated on the two columns alone."""
+    from post_weight_quantization_20_b200.workloads import WORKLOADS
+    wl = WORKLOADS["opt125m"]
+    l = [x for x in wl.layers if x.name == layer][0]
+    X = S.gen_activations(wl.tokens, l.cols, wl.xdtype, wl.xspec, seed=1234, tag=l.tag)
+    H = torch.empty(l.cols, l.cols, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    n = G.gptq_hessian_accumulate(H, 0, to_device(X, wl.xdtype), st)
+    torch.cuda.synchronize()
+    Hg = H.cpu().numpy()
+    assert n == wl.tokens and int(st.item()) == 0
+    g = np.random.default_rng(0)
+    pairs = [(i, i) for i in g.integers(0, l.cols, 16)]
+    pairs += [tuple(sorted(p)) for p in g.integers(0, l.cols, size=(48, 2))]
+    pairs += [(0, l.cols - 1), (l.cols - 1, l.cols - 1), (127, 128), (255, 256)]
+    errs = []
+    for i, j in pairs:
+        Hij, _ = o.hessian(S.to_f64(X[:, [i, j]], wl.xdtype))
+        ref = Hij[0, 1]
+        scale = np.sqrt(Hij[0, 0] * Hij[1, 1])
+        errs.append(abs(Hg[i, j] - ref) / scale)
+    print(f"{layer}: max sampled |dH|/sqrt(HiiHjj) = {max(errs):.2e}")
+    assert max(errs) <= 1e-5, max(errs)
