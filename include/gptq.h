@@ -166,6 +166,31 @@ gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t
 gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits,
                       uint32_t* packed, void* stream);
 
+/*
+ * gptq_prepare_static — gptq_prepare for callers that cannot allocate device memory.
+ * The GPTQ pages have no counterpart to this call; it exists for callers that cannot
+ * allocate where they call us (a plugin inside a framework whose caching allocator
+ * already holds the device memory, code given a fixed memory budget, a service that
+ * must not allocate after start-up because allocation can block and synchronize).
+ * Same arguments, results and device conditions as gptq_prepare, but no `ws`: the
+ * scratch memory is an array of GPTQ_STATIC_SCRATCH_BYTES compiled into the library,
+ * which every GPU that loads the library holds until the process exits.  The call
+ * itself allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
+ *  - cols > GPTQ_STATIC_MAX_COLS returns GPTQ_ERR_WORKSPACE before anything runs;
+ *    use gptq_prepare with a caller workspace for larger layers.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it; make that first
+ *    call before any stream capture.
+ *  - Every call shares the one array, which keeps the previous call's contents (the
+ *    call clears what must start at zero itself).  Calls whose work overlaps on the
+ *    GPU — e.g. on two streams at once — race on the array; order them on one stream
+ *    or synchronize between them.
+ */
+#define GPTQ_STATIC_MAX_COLS 1024
+#define GPTQ_STATIC_SCRATCH_BYTES (12u * 1024u * 1024u)
+gptq_status gptq_prepare_static(const float* H, int64_t cols, const gptq_config* cfg, float* U,
+                                int32_t* perm, int32_t* dev_status, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* gptq_status_string(int status);
 

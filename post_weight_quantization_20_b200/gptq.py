@@ -36,7 +36,9 @@ _DT = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF
 # every symbol include/gptq.h declares
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare",
            "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count",
-           "gptq_last_error")
+           "gptq_last_error", "gptq_prepare_static")
+
+GPTQ_STATIC_MAX_COLS = 1024
 
 
 class GPTQError(RuntimeError):
@@ -86,6 +88,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_status_string.restype = ctypes.c_char_p
     lib.gptq_launch_count.argtypes = []
     lib.gptq_launch_count.restype = ctypes.c_uint64
+    lib.gptq_prepare_static.argtypes = [vp, i64, cfgp, vp, vp, vp, vp]
+    lib.gptq_prepare_static.restype = i32
     lib.gptq_last_error.argtypes = []
     lib.gptq_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -147,6 +151,15 @@ def gptq_prepare(H, cfg, U, perm, ws, status=None, stream=None) -> None:
                                        _ptr(perm), _ptr(ws), ws.numel() * ws.element_size(),
                                        _ptr(status), _stream(stream))
     _check(code, "gptq_prepare")
+
+
+def gptq_prepare_static(H, cfg, U, perm, status=None, stream=None) -> None:
+    """gptq_prepare with the library's built-in scratch array instead of a workspace
+    (for callers that cannot allocate; cols <= GPTQ_STATIC_MAX_COLS)."""
+    _need_cuda(H, U, perm, status)
+    code = load_library().gptq_prepare_static(_ptr(H), H.shape[0], ctypes.byref(cfg), _ptr(U),
+                                              _ptr(perm), _ptr(status), _stream(stream))
+    _check(code, "gptq_prepare_static")
 
 
 def gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws, status=None,
