@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "gemm_f32.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace gptq {
 
@@ -135,56 +136,269 @@ __global__ void k_gather_rev(const float* H, int C, int Cp, const int32_t* perm,
   }
 }
 
-// Unblocked Cholesky of the 64x64 diagonal block at (k0, k0) in shared memory,
-// followed by the inverse of the factor.  Writes the factor back into A (lower,
-// zeros above) and the inverse to T.  A non-positive or non-finite pivot raises
-// GPTQ_ERR_NOT_PD and is replaced by 1 so no NaN spreads.
-__global__ void __launch_bounds__(256)
-k_potrf_diag(float* A, int64_t lda, int k0, float* T, int32_t* st) {
-  __shared__ float S[NB][NB + 1];
-  __shared__ float Ti[NB][NB + 1];
+// ---------------------------------------------------------------------------
+// Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1, by one CTA
+// of 256 threads.
+//   Cholesky: right-looking, one barrier per column.  At step j every thread
+//   reads the pivot, and the threads share the rank-1 update of the trailing
+//   lower triangle, reading the still-unscaled column j; the scaled column goes
+//   to a second tile, so nothing read in the step is written in it.
+//   Inverse: recursive doubling.  With T11, T22 the inverses of the diagonal
+//   sub-blocks of size s, the off-diagonal block is T21 = -T22 (L21 T11); sizes
+//   s = 1, 2, ..., 32 take six levels of small parallel products.
+// ---------------------------------------------------------------------------
+constexpr int LDS = NB + 1;   // padded row of the 64x64 shared tiles
+
+// One level of the recursive-doubling inverse for diagonal sub-blocks of size SZ:
+// for every pair at R0 = 2 b SZ, T21 = -T22 (L21 T11).  Fixed trip counts, no
+// divergent branches: out-of-range terms are masked, not skipped.
+template <int SZ>
+__device__ __forceinline__ void inv_level(const float* S, float* Ti) {
+  constexpr int NOUT = (NB / (2 * SZ)) * SZ * SZ;    // = 32 * SZ outputs
+  constexpr int PER = (NOUT + 255) / 256;
+  const int tid = threadIdx.x;
+  float pv[PER];
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = tid + 256 * u;
+    const int ee = e < NOUT ? e : 0;
+    const int b = ee / (SZ * SZ), rem = ee % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
+    const int R0 = 2 * b * SZ;
+    float acc = 0.f;
+#pragma unroll
+    for (int l = 0; l < SZ; ++l) {
+      const float t = (l >= jj) ? Ti[(R0 + l) * LDS + R0 + jj] : 0.f;   // T11 is lower
+      acc = fmaf(S[(R0 + SZ + i) * LDS + R0 + l], t, acc);
+    }
+    pv[u] = acc;
+  }
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = tid + 256 * u;
+    if (e < NOUT) {
+      const int b = e / (SZ * SZ), rem = e % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
+      Ti[(2 * b * SZ + SZ + i) * LDS + 2 * b * SZ + jj] = pv[u];   // park P in the T21 slot
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = tid + 256 * u;
+    const int ee = e < NOUT ? e : 0;
+    const int b = ee / (SZ * SZ), rem = ee % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
+    const int R0 = 2 * b * SZ;
+    float acc = 0.f;
+#pragma unroll
+    for (int l = 0; l < SZ; ++l) {
+      const float t = (l <= i) ? Ti[(R0 + SZ + i) * LDS + R0 + SZ + l] : 0.f;  // T22 is lower
+      acc = fmaf(t, Ti[(R0 + SZ + l) * LDS + R0 + jj], acc);
+    }
+    pv[u] = -acc;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const int e = tid + 256 * u;
+    if (e < NOUT) {
+      const int b = e / (SZ * SZ), rem = e % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
+      Ti[(2 * b * SZ + SZ + i) * LDS + 2 * b * SZ + jj] = pv[u];
+    }
+  }
+  __syncthreads();
+}
+
+__device__ __noinline__ void diag_factor(float* A, int64_t lda, int k0, float* T, int32_t* st,
+                                         float* S, float* Ti) {
   __shared__ int bad;
   const int tid = threadIdx.x;
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    S[r][c] = A[int64_t(k0 + r) * lda + k0 + c];
+#pragma unroll
+  for (int x = 0; x < (NB * NB) / 256; ++x) {
+    const int e = tid + 256 * x;
+    S[(e >> 6) * LDS + (e & 63)] = A[int64_t(k0 + (e >> 6)) * lda + k0 + (e & 63)];
   }
   if (tid == 0) bad = 0;
   __syncthreads();
-  for (int j = 0; j < NB; ++j) {
-    if (tid == 0) {
-      float p = S[j][j];
-      if (!(p > 0.f) || !isfinite(p)) { bad = 1; p = 1.f; }
-      S[j][j] = sqrtf(p);
+  // Cholesky with the matrix in registers: thread t owns column c = t & 63 at rows
+  // r = (t >> 6) + 4x, x = 0..15.  Step j: the four owners of column j publish it
+  // (double-buffered in the first two rows of Ti), one barrier, then every thread
+  // reads the pivot and the column entries of its rows and updates its registers;
+  // the owners turn their column into L.  Branch-free updates.
+  {
+    const int c = tid & 63, r0 = tid >> 6;
+    float v[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) v[x] = S[(r0 + 4 * x) * LDS + c];
+#pragma unroll 1
+    for (int j = 0; j < NB; ++j) {
+      float* col = Ti + (j & 1) * LDS;
+      if (c == j) {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) col[r0 + 4 * x] = v[x];
+      }
+      __syncthreads();
+      float p = col[j];
+      const bool okp = (p > 0.f) && (p < 3.0e38f);
+      if (!okp && tid == 0) bad = 1;
+      p = okp ? p : 1.f;
+      const float d = __fsqrt_rn(p);
+      const float inv = __frcp_rn(d);
+      const float scj = col[c] * inv * inv;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int r = r0 + 4 * x;
+        const float srj = col[r];
+        const float upd = fmaf(-srj, scj, v[x]);
+        const float own = (r == j) ? d : ((r > j) ? srj * inv : 0.f);
+        v[x] = (c == j) ? own : (((c > j) & (r >= c)) ? upd : v[x]);
+      }
     }
     __syncthreads();
-    const float djj = S[j][j];
-    if (tid > j && tid < NB) S[tid][j] = S[tid][j] / djj;
-    __syncthreads();
-    for (int e = tid; e < NB * NB; e += blockDim.x) {
-      const int r = e / NB, c = e % NB;
-      if (c > j && r >= c) S[r][c] = fmaf(-S[r][j], S[c][j], S[r][c]);
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int r = r0 + 4 * x;
+      S[r * LDS + c] = (c <= r) ? v[x] : 0.f;
     }
     __syncthreads();
   }
-  // inverse of the lower factor, one column per thread (forward substitution)
-  if (tid < NB) {
-    const int c = tid;
-    for (int i = 0; i < c; ++i) Ti[i][c] = 0.f;
-    Ti[c][c] = 1.f / S[c][c];
-    for (int i = c + 1; i < NB; ++i) {
-      float s = 0.f;
-      for (int l = c; l < i; ++l) s = fmaf(S[i][l], Ti[l][c], s);
-      Ti[i][c] = -s / S[i][i];
-    }
+  // Ti <- diag(1 / L_ii)
+#pragma unroll
+  for (int x = 0; x < (NB * NB) / 256; ++x) {
+    const int e = tid + 256 * x;
+    const int r = e >> 6, cc = e & 63;
+    Ti[r * LDS + cc] = (r == cc) ? __frcp_rn(S[r * LDS + r]) : 0.f;
   }
   __syncthreads();
-  for (int e = tid; e < NB * NB; e += blockDim.x) {
-    const int r = e / NB, c = e % NB;
-    A[int64_t(k0 + r) * lda + k0 + c] = (c <= r) ? S[r][c] : 0.f;
-    T[e] = Ti[r][c];
+  inv_level<1>(S, Ti);
+  inv_level<2>(S, Ti);
+  inv_level<4>(S, Ti);
+  inv_level<8>(S, Ti);
+  inv_level<16>(S, Ti);
+  inv_level<32>(S, Ti);
+#pragma unroll
+  for (int x = 0; x < (NB * NB) / 256; ++x) {
+    const int e = tid + 256 * x;
+    const int r = e >> 6, c = e & 63;
+    A[int64_t(k0 + r) * lda + k0 + c] = S[r * LDS + c];
+    T[e] = Ti[r * LDS + c];
   }
   if (tid == 0 && bad) raise_status(st, GPTQ_ERR_NOT_PD);
+}
+
+// ---------------------------------------------------------------------------
+// Persistent factorization + inversion.  One cooperative launch; phases are
+// separated by a grid barrier whose spin is bounded (GPTQ_ERR_TIMEOUT, then
+// every CTA unwinds).  Step k:
+//   phase A: panel L[k0+NB:, k] = A[k0+NB:, k] T_k^T   and   X_k = T_k Bx[k, 0:k0+NB]
+//   phase B: A[k0+NB:, k0+NB:] -= P P^T (lower tiles), Bx[k0+NB:, 0:k0+NB] -= P X_k;
+//            CTA 0 updates the next diagonal block and factors it (lookahead).
+// ---------------------------------------------------------------------------
+struct FactorArgs {
+  float* A;
+  float* Bx;
+  float* T;
+  int lda;
+  int nblk;
+  unsigned* bar;       // monotonically increasing arrival counter (zeroed before launch)
+  int* abort_flag;     // set when a barrier gave up
+  int32_t* status;
+};
+
+constexpr uint32_t BARRIER_SPIN_LIMIT = 1u << 24;
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ bool grid_barrier(const FactorArgs& a, unsigned& epoch) {
+  __shared__ int ok;
+  __syncthreads();
+  ++epoch;
+  if (threadIdx.x == 0) {
+    ok = 1;
+    __threadfence();
+    atomicAdd(a.bar, 1u);
+    const unsigned target = epoch * gridDim.x;
+    uint32_t it = 0;
+    while (ld_acquire(a.bar) < target) {
+      if (++it > BARRIER_SPIN_LIMIT || *(volatile int*)a.abort_flag) {
+        if (atomicExch(a.abort_flag, 1) == 0) raise_status(a.status, GPTQ_ERR_TIMEOUT);
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return ok != 0;
+}
+
+// lower-triangular tile t of an nr x nr tile grid: t = tm (tm + 1) / 2 + tn, tn <= tm
+__device__ __forceinline__ void lower_tile(int t, int& tm, int& tn) {
+  int m = int((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
+  while ((m + 1) * (m + 2) / 2 <= t) ++m;
+  while (m * (m + 1) / 2 > t) --m;
+  tm = m;
+  tn = t - m * (m + 1) / 2;
+}
+
+static_assert(GM_SMEM_FLOATS >= 2 * NB * LDS, "shared buffer holds both diagonal tiles");
+
+__global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs a) {
+  // one buffer: GEMM chunks, or the two 64x64 tiles of the diagonal factor
+  __shared__ __align__(16) float sm[GM_SMEM_FLOATS];
+  float* S = sm;
+  float* Ti = sm + NB * LDS;
+  const int64_t lda = a.lda;
+  unsigned epoch = 0;
+  if (blockIdx.x == 0) diag_factor(a.A, lda, 0, a.T, a.status, S, Ti);
+  if (!grid_barrier(a, epoch)) return;
+  for (int k = 0; k < a.nblk; ++k) {
+    const int k0 = k * NB;
+    const float* Tk = a.T + size_t(k) * NB * NB;
+    const int rest = a.lda - k0 - NB;
+    const int nr = rest / NB;
+    float* panel = a.A + int64_t(k0 + NB) * lda + k0;
+    float* brow = a.Bx + int64_t(k0) * lda;
+    // phase A
+    const GemmProb pan = make_prob(rest, NB, NB, 1.f, panel, lda, 1, Tk, 1, NB, 0.f, panel, lda, 0);
+    const GemmProb xk = make_prob(NB, k0 + NB, NB, 1.f, Tk, NB, 1, brow, lda, 1, 0.f, brow, lda, 0);
+    for (int t = blockIdx.x; t < pan.ntiles + xk.ntiles; t += gridDim.x) {
+      if (t < pan.ntiles) gemm_tile(pan, t, 0, sm);
+      else gemm_tile(xk, 0, t - pan.ntiles, sm);
+    }
+    if (!grid_barrier(a, epoch)) return;
+    if (rest == 0) break;
+    // phase B
+    const GemmProb syrk = make_prob(rest, rest, NB, -1.f, panel, lda, 1, panel, 1, lda, 1.f,
+                                    a.A + int64_t(k0 + NB) * lda + k0 + NB, lda, 1);
+    const GemmProb bup = make_prob(rest, k0 + NB, NB, -1.f, panel, lda, 1, brow, lda, 1, 1.f,
+                                   a.Bx + int64_t(k0 + NB) * lda, lda, 0);
+    const int n_syrk = nr * (nr + 1) / 2;
+    const int n_total = n_syrk + bup.ntiles;
+    if (blockIdx.x == 0) {
+      gemm_tile(syrk, 0, 0, sm);
+      __syncthreads();
+      diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, S, Ti);
+    }
+    const int workers = gridDim.x > 1 ? gridDim.x - 1 : 1;
+    const int first = gridDim.x > 1 ? int(blockIdx.x) - 1 : 0;
+    if (gridDim.x == 1 || blockIdx.x > 0) {
+      for (int t = 1 + first; t < n_total; t += workers) {
+        if (t < n_syrk) {
+          int tm, tn;
+          lower_tile(t, tm, tn);
+          gemm_tile(syrk, tm, tn, sm);
+        } else {
+          const int u = t - n_syrk;
+          gemm_tile(bup, u / bup.tiles_n, u % bup.tiles_n, sm);
+        }
+      }
+    }
+    if (!grid_barrier(a, epoch)) return;
+  }
 }
 
 // U[a][b] = Minv[C-1-a][C-1-b] for a <= b, 0 below the diagonal.
@@ -215,27 +429,27 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
     GPTQ_LAUNCH(k_perm_check, pb, 256, 0, st, L.cnt, C, status);
   }
   const int Cp = L.Cp;
-  const int64_t lda = Cp;
   GPTQ_LAUNCH(k_gather_rev, grid_for(int64_t(Cp) * Cp), 256, 0, st, H, C, Cp, perm, L.lam, L.A,
               L.Bx);
-  for (int k = 0; k < L.nblk; ++k) {
-    const int k0 = k * NB;
-    float* Tk = L.T + size_t(k) * NB * NB;
-    GPTQ_LAUNCH(k_potrf_diag, 1, 256, 0, st, L.A, lda, k0, Tk, status);
-    const int rest = Cp - k0 - NB;
-    float* panel = L.A + int64_t(k0 + NB) * lda + k0;
-    // panel: L[k0+NB:, k-block] = A[k0+NB:, k-block] * T^T
-    GPTQ_TRY(gemm_f32(st, rest, NB, NB, 1.f, panel, lda, 1, Tk, 1, NB, 0.f, panel, lda, 0));
-    // trailing: A[k0+NB:, k0+NB:] -= P P^T (lower tiles)
-    GPTQ_TRY(gemm_f32(st, rest, rest, NB, -1.f, panel, lda, 1, panel, 1, lda, 1.f,
-                      L.A + int64_t(k0 + NB) * lda + k0 + NB, lda, 1));
-    // inverse, block row k: X_k = T * B[k-block, 0:k0+NB]
-    float* brow = L.Bx + int64_t(k0) * lda;
-    GPTQ_TRY(gemm_f32(st, NB, k0 + NB, NB, 1.f, Tk, NB, 1, brow, lda, 1, 0.f, brow, lda, 0));
-    // B[k0+NB:, 0:k0+NB] -= L[k0+NB:, k-block] * X_k
-    GPTQ_TRY(gemm_f32(st, rest, k0 + NB, NB, -1.f, panel, lda, 1, brow, lda, 1, 1.f,
-                      L.Bx + int64_t(k0 + NB) * lda, lda, 0));
-  }
+  // Blocked right-looking Cholesky of A interleaved with the blocked forward
+  // substitution that turns Bx = I into M^-1, in one persistent cooperative launch.
+  unsigned* bar = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(L.lam) + 64);
+  int* abort_flag = reinterpret_cast<int*>(reinterpret_cast<char*>(L.lam) + 128);
+  GPTQ_CUDA(cudaMemsetAsync(reinterpret_cast<char*>(L.lam) + 64, 0, 128, st));
+  FactorArgs fa{L.A, L.Bx, L.T, Cp, L.nblk, bar, abort_flag, status};
+  int per_sm = 0;
+  GPTQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_factor_persistent,
+                                                          GM_THREADS, 0));
+  const int sms = sm_count();
+  if (per_sm <= 0 || sms <= 0) return GPTQ_ERR_CUDA;
+  // enough CTAs for the largest phase, at most what can be co-resident
+  const int nr0 = Cp / NB - 1;
+  const int most = std::max(1, std::max(nr0 * (nr0 + 1) / 2 + nr0, nr0 + Cp / NB));
+  const int grid = std::min(std::min(per_sm, 2) * sms, most + 1);
+  void* args[] = {&fa};
+  GPTQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_factor_persistent), dim3(grid),
+                                        dim3(GM_THREADS), args, 0, st));
+  note_launch();
   GPTQ_LAUNCH(k_write_u, grid_for(int64_t(C) * C), 256, 0, st, L.Bx, Cp, C, U);
   return GPTQ_OK;
 }
