@@ -32,9 +32,12 @@ constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_B * (SW_THREADS / 32)) * 4;
 
 struct QuantLayout {
   float* Wk;
-  float* Err;
+  float* Ehi;
+  float* Elo;
   uint8_t* cp;
   float* lpart;
+  float* Uhi;
+  float* Ulo;
   int tiles;
 };
 
@@ -42,17 +45,21 @@ static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
   QuantLayout L{};
   L.tiles = int((R + SW_ROWS - 1) / SW_ROWS);
   char* p = static_cast<char*>(ws);
-  L.Wk = reinterpret_cast<float*>(p);   p += align256(size_t(R) * C * 4);
-  L.Err = reinterpret_cast<float*>(p);  p += align256(size_t(R) * SW_B * 4);
-  L.cp = reinterpret_cast<uint8_t*>(p); p += align256(size_t(R) * C);
-  L.lpart = reinterpret_cast<float*>(p);
+  L.Wk = reinterpret_cast<float*>(p);    p += align256(size_t(R) * C * 4);
+  L.Ehi = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_B * 4);
+  L.Elo = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_B * 4);
+  L.cp = reinterpret_cast<uint8_t*>(p);  p += align256(size_t(R) * C);
+  L.lpart = reinterpret_cast<float*>(p); p += align256(size_t(L.tiles) * C * 4);
+  L.Uhi = reinterpret_cast<float*>(p);   p += align256(size_t(C) * C * 4);
+  L.Ulo = reinterpret_cast<float*>(p);
   return L;
 }
 
 size_t quantize_ws_bytes(int64_t R, int64_t C, const gptq_config&) {
   const int64_t tiles = (R + SW_ROWS - 1) / SW_ROWS;
-  return align256(size_t(R) * C * 4) + align256(size_t(R) * SW_B * 4) + align256(size_t(R) * C) +
-         align256(size_t(tiles) * C * 4) + 256;
+  return align256(size_t(R) * C * 4) + 2 * align256(size_t(R) * SW_B * 4) +
+         align256(size_t(R) * C) + align256(size_t(tiles) * C * 4) +
+         2 * align256(size_t(C) * C * 4) + 256;
 }
 
 // Grid of a set of values with range [lo, hi] (lo <= 0 <= hi), all in IEEE fp32.
@@ -109,7 +116,8 @@ __global__ void k_row_grid(const float* Wk, int R, int C, int bits, int sym, flo
 // In-panel sweep of columns [i0, i0 + nb) for SW_ROWS rows per CTA.
 __global__ void __launch_bounds__(SW_THREADS)
 k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits, int g, int sym,
-              float* scales, float* zeros, int G, uint8_t* cp, float* Err, float* lpart) {
+              float* scales, float* zeros, int G, uint8_t* cp, float* Ehi, float* Elo,
+              float* lpart) {
   extern __shared__ float sm[];
   float* Us = sm;                       // SW_B x SW_LDU
   float* dinv = Us + SW_B * SW_LDU;     // SW_B
@@ -187,14 +195,18 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
     }
   }
 
-  // errors for the trailing update, codes, and partial column losses
+  // errors for the trailing update (split hi + lo, hi exact in tf32), codes, and
+  // partial column losses
   if (rv) {
-    float* erow = Err + int64_t(r) * SW_B + t * SW_CPT;
+    float* hrow = Ehi + int64_t(r) * SW_B + t * SW_CPT;
+    float* lrow = Elo + int64_t(r) * SW_B + t * SW_CPT;
     uint8_t* crow = cp + int64_t(r) * C + i0 + t * SW_CPT;
 #pragma unroll
     for (int jj = 0; jj < SW_CPT; ++jj) {
       const int col = t * SW_CPT + jj;
-      erow[jj] = e[jj];
+      const float h = __uint_as_float(__float_as_uint(e[jj]) & 0xFFFFE000u);
+      hrow[jj] = h;
+      lrow[jj] = e[jj] - h;
       if (col < nb) crow[jj] = uint8_t((cw[jj >> 2] >> (8 * (jj & 3))) & 0xffu);
     }
   }
@@ -247,7 +259,6 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
                          const float* U, const int32_t* perm, const gptq_config& cfg,
                          uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
                          float* losses, void* ws, int32_t* status) {
-  (void)status;
   QuantLayout L = quant_layout(ws, R, C);
   const int g = cfg.group_size > 0 ? cfg.group_size : 0;
   const int G = g ? (C + g - 1) / g : 1;
@@ -260,15 +271,23 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
   if (!g) {
     GPTQ_LAUNCH(k_row_grid, (R + 7) / 8, 256, 0, st, L.Wk, R, C, cfg.bits, cfg.sym, scales, zeros);
   }
+  const bool tc = C > SW_B && trailing_tc_supported(C);
+  if (tc) GPTQ_TRY(split_tf32_t(st, U, C, L.Uhi, L.Ulo));
   for (int i0 = 0; i0 < C; i0 += SW_B) {
     const int nb = min(SW_B, C - i0);
     GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
-                g, cfg.sym, scales, zeros, G, L.cp, L.Err, L.lpart);
+                g, cfg.sym, scales, zeros, G, L.cp, L.Ehi, L.Elo, L.lpart);
     const int e = i0 + nb;
     if (e < C) {
       // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]
-      GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Err, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
-                        1.f, L.Wk + e, C, 0));
+      if (tc) {
+        GPTQ_TRY(trailing_update_tc(st, L.Wk, R, C, i0, e, L.Ehi, L.Elo, L.Uhi, L.Ulo, status));
+      } else {
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Ehi, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
+                          1.f, L.Wk + e, C, 0));
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Elo, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
+                          1.f, L.Wk + e, C, 0));
+      }
     }
   }
   GPTQ_LAUNCH(k_scatter_codes, grid_for(int64_t(R) * C), 256, 0, st, L.cp, R, C, perm, codes);

@@ -197,6 +197,8 @@ CASES = [
     ("8b-row", 64, 160, 2000, S.F32, S.F16, 8, 0, False, False, S.ActSpec()),
     ("single-col", 50, 1, 500, S.F32, S.F32, 4, 0, False, False, S.ActSpec()),
     ("single-row", 1, 300, 2000, S.F16, S.F16, 4, 128, False, True, S.ActSpec(mix_rank=3)),
+    ("C203-fallback-paths", 70, 203, 1500, S.F16, S.F16, 4, 0, False, False, S.ActSpec(mix_rank=5)),
+    ("tall-1000x640", 1000, 640, 3000, S.BF16, S.BF16, 4, 128, False, True, S.ActSpec(mix_rank=8)),
 ]
 
 
