@@ -240,8 +240,11 @@ __device__ __noinline__ void diag_factor(float* A, int64_t lda, int k0, float* T
       const bool okp = (p > 0.f) && (p < 3.0e38f);
       if (!okp && tid == 0) bad = 1;
       p = okp ? p : 1.f;
-      const float d = __fsqrt_rn(p);
-      const float inv = __frcp_rn(d);
+      // 1/sqrt(p): hardware estimate refined by one Newton step (a short chain
+      // compared with an IEEE square root followed by an IEEE reciprocal)
+      const float y0 = rsqrtf(p);
+      const float inv = y0 * fmaf(-0.5f * p * y0, y0, 1.5f);
+      const float d = p * inv;
       const float scj = col[c] * inv * inv;
 #pragma unroll
       for (int x = 0; x < 16; ++x) {

@@ -23,12 +23,13 @@
 namespace gptq {
 
 constexpr int SW_B = 128;                 // panel width (columns)
-constexpr int SW_TPR = 4;                 // threads per row
-constexpr int SW_CPT = SW_B / SW_TPR;     // panel columns owned by one thread
-constexpr int SW_ROWS = 32;               // rows per CTA
+constexpr int SW_TPR = 8;                 // threads per row
+constexpr int SW_CPT = SW_B / SW_TPR;     // panel columns owned by one thread (16)
+constexpr int SW_ROWS = 16;               // rows per CTA
 constexpr int SW_THREADS = SW_ROWS * SW_TPR;
 constexpr int SW_LDU = SW_B + 4 * SW_TPR; // skewed U row: column c at c + 4*(c / SW_CPT)
-constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_B * (SW_THREADS / 32)) * 4;
+// U block, 1/U_qq, per-row losses of the panel
+constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_ROWS * SW_B) * 4;
 
 struct QuantLayout {
   float* Wk;
@@ -113,34 +114,58 @@ __global__ void k_row_grid(const float* Wk, int R, int C, int bits, int sym, flo
   }
 }
 
-// In-panel sweep of columns [i0, i0 + nb) for SW_ROWS rows per CTA.
+// In-panel sweep of columns [i0, i0 + nb) for SW_ROWS rows per CTA.  Thread
+// (row, t) owns panel columns 16t .. 16t + 15 of its row in registers.
+__device__ __forceinline__ int uskew(int b) { return b + 4 * (b / SW_CPT); }
+
 __global__ void __launch_bounds__(SW_THREADS)
 k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits, int g, int sym,
               float* scales, float* zeros, int G, uint8_t* cp, float* Ehi, float* Elo,
               float* lpart) {
-  extern __shared__ float sm[];
+  extern __shared__ __align__(16) float sm[];
   float* Us = sm;                       // SW_B x SW_LDU
   float* dinv = Us + SW_B * SW_LDU;     // SW_B
-  float* red = dinv + SW_B;             // warps x SW_B
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t = tid % SW_TPR;
-  const int r = blockIdx.x * SW_ROWS + tid / SW_TPR;
+  float* lrow = dinv + SW_B;            // SW_ROWS x SW_B
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int t = tid % SW_TPR, rl = tid / SW_TPR;
+  const int r = blockIdx.x * SW_ROWS + rl;
   const bool rv = r < R;
-  for (int e = tid; e < SW_B * SW_B; e += SW_THREADS) {
-    const int a = e / SW_B, b = e % SW_B;
-    const float v = (a < nb && b < nb) ? U[int64_t(i0 + a) * C + i0 + b] : 0.f;
-    Us[a * SW_LDU + b + 4 * (b / SW_CPT)] = v;
+  // U block (rows and columns i0 .. i0 + nb) into the skewed layout, 16-byte loads
+  const bool vec = ((C & 3) == 0) && (nb == SW_B) && ((reinterpret_cast<uintptr_t>(U) & 15) == 0);
+  if (vec) {
+#pragma unroll 8
+    for (int x = 0; x < (SW_B * SW_B / 4) / SW_THREADS; ++x) {
+      const int e4 = tid + SW_THREADS * x;
+      const int a = e4 / (SW_B / 4), b = 4 * (e4 % (SW_B / 4));
+      const float4 v = *reinterpret_cast<const float4*>(U + int64_t(i0 + a) * C + i0 + b);
+      *reinterpret_cast<float4*>(Us + a * SW_LDU + uskew(b)) = v;
+    }
+  } else {
+    for (int e = tid; e < SW_B * SW_B; e += SW_THREADS) {
+      const int a = e / SW_B, b = e % SW_B;
+      Us[a * SW_LDU + uskew(b)] = (a < nb && b < nb) ? U[int64_t(i0 + a) * C + i0 + b] : 0.f;
+    }
   }
   if (tid < SW_B) dinv[tid] = tid < nb ? 1.f / U[int64_t(i0 + tid) * C + i0 + tid] : 0.f;
   float w[SW_CPT];
   const float* wrow = Wk + int64_t(rv ? r : 0) * C + i0 + t * SW_CPT;
+  if (rv && vec) {
 #pragma unroll
-  for (int jj = 0; jj < SW_CPT; ++jj) w[jj] = (rv && t * SW_CPT + jj < nb) ? wrow[jj] : 0.f;
+    for (int q = 0; q < SW_CPT / 4; ++q) {
+      const float4 v = *reinterpret_cast<const float4*>(wrow + 4 * q);
+      w[4 * q] = v.x; w[4 * q + 1] = v.y; w[4 * q + 2] = v.z; w[4 * q + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int jj = 0; jj < SW_CPT; ++jj) w[jj] = (rv && t * SW_CPT + jj < nb) ? wrow[jj] : 0.f;
+  }
   __syncthreads();
 
   const float maxq = float((1 << bits) - 1);
   float s = 1.f, z = 0.f;
   if (g <= 0 && rv) { s = scales[r]; z = zeros[r]; }
+  float inv_s = __frcp_rn(s), cmin = -z, cmax = maxq - z;
+  const int gmask = g - 1;   // g divides 128, so it is a power of two
   float e[SW_CPT];
   uint32_t cw[SW_CPT / 4];
 #pragma unroll
@@ -153,7 +178,7 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
     for (int qq = 0; qq < SW_CPT; ++qq) {
       const int q = c * SW_CPT + qq;
       if (q >= nb) break;
-      if (g > 0 && (q % g) == 0) {
+      if (g > 0 && (q & gmask) == 0) {
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int jj = 0; jj < SW_CPT; ++jj) {
@@ -169,19 +194,25 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
           hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
         }
         grid_params(lo, hi, maxq, sym, s, z);
+        inv_s = __frcp_rn(s);
+        cmin = -z;
+        cmax = maxq - z;
         if (t == 0 && rv) {
           const int gi = (i0 + q) / g;
           scales[int64_t(r) * G + gi] = s;
           zeros[int64_t(r) * G + gi] = z;
         }
       }
+      // code - z = clamp(rint(x / s), -z, maxq - z), with x / s taken as x * (1/s)
+      // (within 2 ulp of the division); err = (x - s (code - z)) / U_qq, where the
+      // fma rounds x - s (code - z) once
+      const float dq = dinv[q];
       const float x = __shfl_sync(0xffffffffu, w[qq], (lane & ~(SW_TPR - 1)) | c);
-      const float code = fminf(fmaxf(rintf(__fdiv_rn(x, s)) + z, 0.f), maxq);
-      const float Q = s * (code - z);
-      const float err = (x - Q) * dinv[q];
+      const float cq = fminf(fmaxf(rintf(x * inv_s), cmin), cmax);
+      const float err = fmaf(-s, cq, x) * dq;
       if (t == c) {
         e[qq] = err;
-        cw[qq >> 2] |= uint32_t(code) << (8 * (qq & 3));
+        cw[qq >> 2] |= uint32_t(cq + z) << (8 * (qq & 3));
       }
       const float* urow = Us + q * SW_LDU + t * (SW_CPT + 4);
 #pragma unroll
@@ -196,33 +227,37 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
   }
 
   // errors for the trailing update (split hi + lo, hi exact in tf32), codes, and
-  // partial column losses
+  // per-row losses for the column reduction
   if (rv) {
-    float* hrow = Ehi + int64_t(r) * SW_B + t * SW_CPT;
-    float* lrow = Elo + int64_t(r) * SW_B + t * SW_CPT;
-    uint8_t* crow = cp + int64_t(r) * C + i0 + t * SW_CPT;
+    float hv[SW_CPT], lv[SW_CPT];
 #pragma unroll
     for (int jj = 0; jj < SW_CPT; ++jj) {
-      const int col = t * SW_CPT + jj;
-      const float h = __uint_as_float(__float_as_uint(e[jj]) & 0xFFFFE000u);
-      hrow[jj] = h;
-      lrow[jj] = e[jj] - h;
-      if (col < nb) crow[jj] = uint8_t((cw[jj >> 2] >> (8 * (jj & 3))) & 0xffu);
+      hv[jj] = __uint_as_float(__float_as_uint(e[jj]) & 0xFFFFE000u);
+      lv[jj] = e[jj] - hv[jj];
+    }
+    float4* hrow = reinterpret_cast<float4*>(Ehi + int64_t(r) * SW_B + t * SW_CPT);
+    float4* lrw = reinterpret_cast<float4*>(Elo + int64_t(r) * SW_B + t * SW_CPT);
+#pragma unroll
+    for (int q = 0; q < SW_CPT / 4; ++q) {
+      hrow[q] = make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
+      lrw[q] = make_float4(lv[4 * q], lv[4 * q + 1], lv[4 * q + 2], lv[4 * q + 3]);
+    }
+    uint8_t* crow = cp + int64_t(r) * C + i0 + t * SW_CPT;
+    if (vec && ((reinterpret_cast<uintptr_t>(crow) & 15) == 0)) {
+      *reinterpret_cast<uint4*>(crow) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    } else {
+#pragma unroll
+      for (int jj = 0; jj < SW_CPT; ++jj)
+        if (t * SW_CPT + jj < nb) crow[jj] = uint8_t((cw[jj >> 2] >> (8 * (jj & 3))) & 0xffu);
     }
   }
 #pragma unroll
-  for (int jj = 0; jj < SW_CPT; ++jj) {
-    float l = rv ? 0.5f * e[jj] * e[jj] : 0.f;
-    l += __shfl_xor_sync(0xffffffffu, l, 4);
-    l += __shfl_xor_sync(0xffffffffu, l, 8);
-    l += __shfl_xor_sync(0xffffffffu, l, 16);
-    if (lane < SW_TPR) red[warp * SW_B + t * SW_CPT + jj] = l;
-  }
+  for (int jj = 0; jj < SW_CPT; ++jj) lrow[rl * SW_B + t * SW_CPT + jj] = rv ? 0.5f * e[jj] * e[jj] : 0.f;
   __syncthreads();
   if (tid < nb) {
     float l = 0.f;
 #pragma unroll
-    for (int wi = 0; wi < SW_THREADS / 32; ++wi) l += red[wi * SW_B + tid];
+    for (int i = 0; i < SW_ROWS; ++i) l += lrow[i * SW_B + tid];
     lpart[int64_t(blockIdx.x) * C + i0 + tid] = l;
   }
 }

@@ -56,7 +56,11 @@ def compare_layer(W64, H64, n, perm, gpu, bits, group, sym, tau, damp=0.01, bloc
     scale_rel = float(np.max(np.abs(s_o - s_g) / np.maximum(np.abs(s_o), 1e-30))) if s_o.size else 0.0
     zero_diff = float(np.max(np.abs(ref["zeros"] - gpu["zeros"]))) if s_o.size else 0.0
     lo, lg = ref["losses"], gpu["losses"].astype(np.float64)
-    loss_rel = float(np.sum(np.abs(lo - lg)) / max(np.sum(np.abs(lo)), 1e-300))
+    # floor: a millionth of the loss of quantizing every weight to zero, so that
+    # layers whose weights sit on the grid (losses at rounding level) compare sanely
+    U = ref["U"]
+    zero_loss = float(np.sum(np.sum(ref["Wp"] ** 2, axis=0) / (2.0 * np.diag(U) ** 2))) if R else 0.0
+    loss_rel = float(np.sum(np.abs(lo - lg)) / max(np.sum(np.abs(lo)), 1e-6 * zero_loss, 1e-300))
     Qg = gpu["scales"][:, gpu["g_idx"]].astype(np.float64) * \
         (gpu["codes"].astype(np.float64) - gpu["zeros"][:, gpu["g_idx"]].astype(np.float64))
     rg = o.reconstruction_error(W64, Qg, H64, n)
