@@ -80,50 +80,88 @@ def gen_inputs(wl, seed=1234):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock and clock-event reasons of one GPU, sampled while a region runs.
+
+    NVML is polled from a thread every few milliseconds (the timed regions are
+    tens of milliseconds); without NVML, nvidia-smi is run in the background.
+    The device is matched by PCI bus id, so CUDA_VISIBLE_DEVICES does not matter.
+    """
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, device):
+        import torch
+        pr = torch.cuda.get_device_properties(device)
+        self.bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+        self.rows = []
+        self.thread = None
         self.proc = None
         self.path = None
+        self.stop_evt = None
+
+    def _nvml_loop(self, nv, h):
+        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.stop_evt.is_set():
+            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            self.rows.append((float(sm), float(mx), [k for k, b in bits.items() if rs & b]))
+            self.stop_evt.wait(self.PERIOD_S)
 
     def start(self):
+        import threading
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(self.bus.encode())
+            self.stop_evt = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.bus}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            rows = self.rows
+        elif self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            rows = []
+            with open(self.path) as f:
+                for line in f:
+                    r = [p.strip() for p in line.split(",")]
+                    if len(r) >= 9 and r[1].replace(".", "").isdigit():
+                        rows.append((float(r[1]), float(r[2]) if r[2].replace(".", "").isdigit() else 0.0,
+                                     [names[i] for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]]))
+            os.unlink(self.path)
+        else:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
-                          and "Not" not in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted({x for r in rows for x in r[2]}), "samples": len(rows)}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -201,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
         if st:
             raise RuntimeError(f"device status {G.status_names(st)}")
 
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(dev)
     barrier()
     torch.cuda.synchronize(dev)
     clocks.start()

@@ -137,154 +137,144 @@ __global__ void k_gather_rev(const float* H, int C, int Cp, const int32_t* perm,
 }
 
 // ---------------------------------------------------------------------------
-// Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1, by one CTA
-// of 256 threads.
-//   Cholesky: right-looking, one barrier per column.  At step j every thread
-//   reads the pivot, and the threads share the rank-1 update of the trailing
-//   lower triangle, reading the still-unscaled column j; the scaled column goes
-//   to a second tile, so nothing read in the step is written in it.
-//   Inverse: recursive doubling.  With T11, T22 the inverses of the diagonal
-//   sub-blocks of size s, the off-diagonal block is T21 = -T22 (L21 T11); sizes
-//   s = 1, 2, ..., 32 take six levels of small parallel products.
+// Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1, by four
+// warps holding the block in registers (the CTA only stages it in and out).
+//
+// Warps 0-1 factor: thread c holds column c.  At step j the owner of column j has
+// published it to shared memory; every thread forms 1/sqrt(pivot) itself, threads
+// c > j apply the rank-1 update A[:, c] -= L[:, j] L[c][j] to their column as
+// A[:, c] -= A[:, j] (A[c][j] / pivot), and column j, scaled, is written out as
+// L[:, j].  The owner of column j+1 publishes it when its update is done.
+// Warps 2-3 invert, one step behind: thread r holds row r of the forward
+// substitution L B = I, and step i subtracts (L[r][i] / L[i][i]) B[i][:] from rows
+// r > i, with row B[i][:] published by its owner; finally T[r][:] = B[r][:] / L[r][r].
+// Every register index is static (a thread's column or row is its own), the loop
+// body is short, and the steps are separated by one 128-thread barrier.  Entries
+// above the diagonal hold scratch values that are never read; the outputs are
+// masked to the lower triangle.
 // ---------------------------------------------------------------------------
 constexpr int LDS = NB + 1;   // padded row of the 64x64 shared tiles
+constexpr int DF_BCAST = 2 * NB * LDS;                 // broadcast area after the two tiles
+static_assert(GM_SMEM_FLOATS >= DF_BCAST + 5 * NB, "shared buffer holds the broadcasts");
 
-// One level of the recursive-doubling inverse for diagonal sub-blocks of size SZ:
-// for every pair at R0 = 2 b SZ, T21 = -T22 (L21 T11).  Fixed trip counts, no
-// divergent branches: out-of-range terms are masked, not skipped.
-template <int SZ>
-__device__ __forceinline__ void inv_level(const float* S, float* Ti) {
-  constexpr int NOUT = (NB / (2 * SZ)) * SZ * SZ;    // = 32 * SZ outputs
-  constexpr int PER = (NOUT + 255) / 256;
-  const int tid = threadIdx.x;
-  float pv[PER];
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int e = tid + 256 * u;
-    const int ee = e < NOUT ? e : 0;
-    const int b = ee / (SZ * SZ), rem = ee % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
-    const int R0 = 2 * b * SZ;
-    float acc = 0.f;
-#pragma unroll
-    for (int l = 0; l < SZ; ++l) {
-      const float t = (l >= jj) ? Ti[(R0 + l) * LDS + R0 + jj] : 0.f;   // T11 is lower
-      acc = fmaf(S[(R0 + SZ + i) * LDS + R0 + l], t, acc);
-    }
-    pv[u] = acc;
-  }
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int e = tid + 256 * u;
-    if (e < NOUT) {
-      const int b = e / (SZ * SZ), rem = e % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
-      Ti[(2 * b * SZ + SZ + i) * LDS + 2 * b * SZ + jj] = pv[u];   // park P in the T21 slot
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int e = tid + 256 * u;
-    const int ee = e < NOUT ? e : 0;
-    const int b = ee / (SZ * SZ), rem = ee % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
-    const int R0 = 2 * b * SZ;
-    float acc = 0.f;
-#pragma unroll
-    for (int l = 0; l < SZ; ++l) {
-      const float t = (l <= i) ? Ti[(R0 + SZ + i) * LDS + R0 + SZ + l] : 0.f;  // T22 is lower
-      acc = fmaf(t, Ti[(R0 + SZ + l) * LDS + R0 + jj], acc);
-    }
-    pv[u] = -acc;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int u = 0; u < PER; ++u) {
-    const int e = tid + 256 * u;
-    if (e < NOUT) {
-      const int b = e / (SZ * SZ), rem = e % (SZ * SZ), i = rem / SZ, jj = rem % SZ;
-      Ti[(2 * b * SZ + SZ + i) * LDS + 2 * b * SZ + jj] = pv[u];
-    }
-  }
-  __syncthreads();
+__device__ __forceinline__ void df_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+// 1/sqrt(p): hardware estimate refined by one Newton step
+__device__ __forceinline__ float rsqrt_nr(float p) {
+  const float y0 = rsqrtf(p);
+  return y0 * fmaf(-0.5f * p * y0, y0, 1.5f);
 }
 
-__device__ __noinline__ void diag_factor(float* A, int64_t lda, int k0, float* T, int32_t* st,
-                                         float* S, float* Ti) {
-  __shared__ int bad;
+// S: the block on entry, L on exit.  Ti: T on exit.  bc: 5 * NB floats.
+__device__ __forceinline__ void quad_factor(float* S, float* Ti, float* bc, int32_t* st,
+                                            const int tid) {
+  float* colb = bc;               // [2][NB]: column j of the trailing matrix
+  float* rowb = bc + 2 * NB;      // [2][NB]: row i of B
+  float* sinv = bc + 4 * NB;      // [NB]: 1 / L[j][j]
+  float v[NB];
+  if (tid < NB) {
+    const int c = tid;
+#pragma unroll
+    for (int r = 0; r < NB; ++r) v[r] = S[r * LDS + c];
+    colb[c] = S[c * LDS];         // column 0 (symmetric: row 0)
+  } else {
+    const int r = tid - NB;
+#pragma unroll
+    for (int c = 0; c < NB; ++c) v[c] = (c == r) ? 1.f : 0.f;
+    rowb[r] = (r == 0) ? 1.f : 0.f;
+  }
+  bool bad = false;
+  df_bar();
+#pragma unroll 1
+  for (int j = 0; j <= NB; ++j) {
+    if (tid < NB) {
+      if (j < NB) {
+        const int c = tid;
+        const float* col = colb + (j & 1) * NB;
+        float p = col[j];
+        const bool okp = (p > 0.f) && (p < 3.0e38f);
+        bad |= (c == 0) && !okp;
+        p = okp ? p : 1.f;
+        const float inv = rsqrt_nr(p);
+        const float cc = col[c];
+        S[c * LDS + j] = (c > j) ? cc * inv : ((c == j) ? p * inv : 0.f);
+        if (c == 0) sinv[j] = inv;
+        if (c > j) {
+          const float sc = cc * inv * inv;
+#pragma unroll
+          for (int q = 0; q < NB / 4; ++q) {
+            const float4 x = *reinterpret_cast<const float4*>(col + 4 * q);
+            v[4 * q + 0] = fmaf(-x.x, sc, v[4 * q + 0]);
+            v[4 * q + 1] = fmaf(-x.y, sc, v[4 * q + 1]);
+            v[4 * q + 2] = fmaf(-x.z, sc, v[4 * q + 2]);
+            v[4 * q + 3] = fmaf(-x.w, sc, v[4 * q + 3]);
+          }
+          if (c == j + 1) {
+            float* nx = colb + ((j + 1) & 1) * NB;
+#pragma unroll
+            for (int q = 0; q < NB / 4; ++q)
+              *reinterpret_cast<float4*>(nx + 4 * q) =
+                  make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+        }
+      }
+    } else if (j >= 1) {
+      // inverse step i = j - 1 (needs L[:, i] and 1/L[i][i], written in step i)
+      const int r = tid - NB, i = j - 1;
+      if (r > i) {
+        const float k = S[r * LDS + i] * sinv[i];
+        const float* row = rowb + (i & 1) * NB;
+#pragma unroll
+        for (int q = 0; q < NB / 4; ++q) {
+          const float4 x = *reinterpret_cast<const float4*>(row + 4 * q);
+          v[4 * q + 0] = fmaf(-k, x.x, v[4 * q + 0]);
+          v[4 * q + 1] = fmaf(-k, x.y, v[4 * q + 1]);
+          v[4 * q + 2] = fmaf(-k, x.z, v[4 * q + 2]);
+          v[4 * q + 3] = fmaf(-k, x.w, v[4 * q + 3]);
+        }
+        if (r == i + 1) {
+          float* nx = rowb + ((i + 1) & 1) * NB;
+#pragma unroll
+          for (int q = 0; q < NB / 4; ++q)
+            *reinterpret_cast<float4*>(nx + 4 * q) =
+                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      }
+    }
+    df_bar();
+  }
+  if (tid >= NB) {
+    const int r = tid - NB;
+    const float ir = sinv[r];
+#pragma unroll
+    for (int c = 0; c < NB; ++c) Ti[r * LDS + c] = (c <= r) ? v[c] * ir : 0.f;
+  }
+  if (bad) raise_status(st, GPTQ_ERR_NOT_PD);
+}
+
+// Factor the diagonal block at (k0, k0) of A in place (L, zeros above the
+// diagonal) and write T = L^-1 (64x64, row-major).  Called by all GM_THREADS
+// threads of the CTA with sm = GM_SMEM_FLOATS floats of shared memory.
+__device__ __forceinline__ void diag_factor(float* A, int64_t lda, int k0, float* T, int32_t* st,
+                                         float* sm) {
+  float* S = sm;
+  float* Ti = sm + NB * LDS;
   const int tid = threadIdx.x;
 #pragma unroll
-  for (int x = 0; x < (NB * NB) / 256; ++x) {
-    const int e = tid + 256 * x;
+  for (int x = 0; x < (NB * NB) / GM_THREADS; ++x) {
+    const int e = tid + GM_THREADS * x;
     S[(e >> 6) * LDS + (e & 63)] = A[int64_t(k0 + (e >> 6)) * lda + k0 + (e & 63)];
   }
-  if (tid == 0) bad = 0;
   __syncthreads();
-  // Cholesky with the matrix in registers: thread t owns column c = t & 63 at rows
-  // r = (t >> 6) + 4x, x = 0..15.  Step j: the four owners of column j publish it
-  // (double-buffered in the first two rows of Ti), one barrier, then every thread
-  // reads the pivot and the column entries of its rows and updates its registers;
-  // the owners turn their column into L.  Branch-free updates.
-  {
-    const int c = tid & 63, r0 = tid >> 6;
-    float v[16];
-#pragma unroll
-    for (int x = 0; x < 16; ++x) v[x] = S[(r0 + 4 * x) * LDS + c];
-#pragma unroll 1
-    for (int j = 0; j < NB; ++j) {
-      float* col = Ti + (j & 1) * LDS;
-      if (c == j) {
-#pragma unroll
-        for (int x = 0; x < 16; ++x) col[r0 + 4 * x] = v[x];
-      }
-      __syncthreads();
-      float p = col[j];
-      const bool okp = (p > 0.f) && (p < 3.0e38f);
-      if (!okp && tid == 0) bad = 1;
-      p = okp ? p : 1.f;
-      // 1/sqrt(p): hardware estimate refined by one Newton step (a short chain
-      // compared with an IEEE square root followed by an IEEE reciprocal)
-      const float y0 = rsqrtf(p);
-      const float inv = y0 * fmaf(-0.5f * p * y0, y0, 1.5f);
-      const float d = p * inv;
-      const float scj = col[c] * inv * inv;
-#pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        const int r = r0 + 4 * x;
-        const float srj = col[r];
-        const float upd = fmaf(-srj, scj, v[x]);
-        const float own = (r == j) ? d : ((r > j) ? srj * inv : 0.f);
-        v[x] = (c == j) ? own : (((c > j) & (r >= c)) ? upd : v[x]);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int x = 0; x < 16; ++x) {
-      const int r = r0 + 4 * x;
-      S[r * LDS + c] = (c <= r) ? v[x] : 0.f;
-    }
-    __syncthreads();
-  }
-  // Ti <- diag(1 / L_ii)
-#pragma unroll
-  for (int x = 0; x < (NB * NB) / 256; ++x) {
-    const int e = tid + 256 * x;
-    const int r = e >> 6, cc = e & 63;
-    Ti[r * LDS + cc] = (r == cc) ? __frcp_rn(S[r * LDS + r]) : 0.f;
-  }
+  if (tid < 2 * NB) quad_factor(S, Ti, sm + DF_BCAST, st, tid);
   __syncthreads();
-  inv_level<1>(S, Ti);
-  inv_level<2>(S, Ti);
-  inv_level<4>(S, Ti);
-  inv_level<8>(S, Ti);
-  inv_level<16>(S, Ti);
-  inv_level<32>(S, Ti);
 #pragma unroll
-  for (int x = 0; x < (NB * NB) / 256; ++x) {
-    const int e = tid + 256 * x;
+  for (int x = 0; x < (NB * NB) / GM_THREADS; ++x) {
+    const int e = tid + GM_THREADS * x;
     const int r = e >> 6, c = e & 63;
     A[int64_t(k0 + r) * lda + k0 + c] = S[r * LDS + c];
     T[e] = Ti[r * LDS + c];
   }
-  if (tid == 0 && bad) raise_status(st, GPTQ_ERR_NOT_PD);
 }
 
 // ---------------------------------------------------------------------------
@@ -347,16 +337,12 @@ __device__ __forceinline__ void lower_tile(int t, int& tm, int& tn) {
   tn = t - m * (m + 1) / 2;
 }
 
-static_assert(GM_SMEM_FLOATS >= 2 * NB * LDS, "shared buffer holds both diagonal tiles");
-
 __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs a) {
-  // one buffer: GEMM chunks, or the two 64x64 tiles of the diagonal factor
+  // one buffer: GEMM chunks, or the tiles of the diagonal factor
   __shared__ __align__(16) float sm[GM_SMEM_FLOATS];
-  float* S = sm;
-  float* Ti = sm + NB * LDS;
   const int64_t lda = a.lda;
   unsigned epoch = 0;
-  if (blockIdx.x == 0) diag_factor(a.A, lda, 0, a.T, a.status, S, Ti);
+  if (blockIdx.x == 0) diag_factor(a.A, lda, 0, a.T, a.status, sm);
   if (!grid_barrier(a, epoch)) return;
   for (int k = 0; k < a.nblk; ++k) {
     const int k0 = k * NB;
@@ -384,7 +370,7 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
     if (blockIdx.x == 0) {
       gemm_tile(syrk, 0, 0, sm);
       __syncthreads();
-      diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, S, Ti);
+      diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, sm);
     }
     const int workers = gridDim.x > 1 ? gridDim.x - 1 : 1;
     const int first = gridDim.x > 1 ? int(blockIdx.x) - 1 : 0;
