@@ -137,27 +137,38 @@ __global__ void k_gather_rev(const float* H, int C, int Cp, const int32_t* perm,
 }
 
 // ---------------------------------------------------------------------------
-// Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1, by four
-// warps holding the block in registers (the CTA only stages it in and out).
+// Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1 by one CTA
+// holding the block in registers, four columns per step.
 //
-// Warps 0-1 factor: thread c holds column c.  At step j the owner of column j has
-// published it to shared memory; every thread forms 1/sqrt(pivot) itself, threads
-// c > j apply the rank-1 update A[:, c] -= L[:, j] L[c][j] to their column as
-// A[:, c] -= A[:, j] (A[c][j] / pivot), and column j, scaled, is written out as
-// L[:, j].  The owner of column j+1 publishes it when its update is done.
-// Warps 2-3 invert, one step behind: thread r holds row r of the forward
-// substitution L B = I, and step i subtracts (L[r][i] / L[i][i]) B[i][:] from rows
-// r > i, with row B[i][:] published by its owner; finally T[r][:] = B[r][:] / L[r][r].
-// Every register index is static (a thread's column or row is its own), the loop
-// body is short, and the steps are separated by one 128-thread barrier.  Entries
-// above the diagonal hold scratch values that are never read; the outputs are
-// masked to the lower triangle.
+// Warps 0-3 factor: thread (c, h) holds rows 32h .. 32h+31 of column c of the
+// trailing matrix.  At block step b (columns j0 = 4b .. j0+3) the owners of those
+// columns have published them, P (64 x 4, P[r][q] = A[r][j0+q]).  Every thread
+// factors the 4x4 pivot block P1 = L11 L11^T itself and forms M = L11^-1 and
+// W = P1^-1 = M^T M.  Then, with p_c = P[c][:] the own row of P,
+//   L[c][j0..j0+3] = M p_c               (this is L11's row for c in the block)
+//   A[:, c]       -= P (W p_c)           (c > j0+3: the rank-4 trailing update)
+// and the owners of the next four columns publish them.
+// Warps 4-7 invert, one block step behind: thread (r, h) holds columns
+// 32h .. 32h+31 of row r of the forward substitution L B = I.  With B_blk the four
+// published rows j0..j0+3,
+//   B[r] -= (W p_r)^T B_blk                    for r > j0+3,
+//   B[r] -= (e_{r-j0} - M[r-j0][:])^T B_blk   for r in the block,
+// which leaves T = L^-1 in the rows when the last block is done.  The factor
+// threads hand the coefficient vectors over through shared memory.
+// Every register index is static, the loop body is short, and block steps are
+// separated by one CTA barrier.  Entries above the diagonal hold scratch values
+// that are never read; the outputs are masked to the lower triangle.
 // ---------------------------------------------------------------------------
 constexpr int LDS = NB + 1;   // padded row of the 64x64 shared tiles
-constexpr int DF_BCAST = 2 * NB * LDS;                 // broadcast area after the two tiles
-static_assert(GM_SMEM_FLOATS >= DF_BCAST + 5 * NB, "shared buffer holds the broadcasts");
-
-__device__ __forceinline__ void df_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+constexpr int KB = 4;         // columns per block step
+constexpr int NSTEP = NB / KB;
+constexpr int HR = NB / 2;    // rows (or columns) per thread
+// broadcasts P [2][KB][NB], Bp [2][KB][NB], cw [2][NB][KB]; they live in the T
+// tile, which is written only after the last step
+constexpr int DF_BCAST_FLOATS = 3 * 2 * KB * NB;
+static_assert(DF_BCAST_FLOATS <= NB * LDS, "the T tile holds the broadcasts");
+static_assert((NB * LDS) % 4 == 0, "the T tile is 16-byte aligned");
+static_assert(GM_THREADS == 4 * NB, "two roles x two halves x NB threads");
 
 // 1/sqrt(p): hardware estimate refined by one Newton step
 __device__ __forceinline__ float rsqrt_nr(float p) {
@@ -165,89 +176,154 @@ __device__ __forceinline__ float rsqrt_nr(float p) {
   return y0 * fmaf(-0.5f * p * y0, y0, 1.5f);
 }
 
-// S: the block on entry, L on exit.  Ti: T on exit.  bc: 5 * NB floats.
-__device__ __forceinline__ void quad_factor(float* S, float* Ti, float* bc, int32_t* st,
-                                            const int tid) {
-  float* colb = bc;               // [2][NB]: column j of the trailing matrix
-  float* rowb = bc + 2 * NB;      // [2][NB]: row i of B
-  float* sinv = bc + 4 * NB;      // [NB]: 1 / L[j][j]
-  float v[NB];
-  if (tid < NB) {
-    const int c = tid;
+// 1/sqrt of a pivot; a pivot that is not positive and finite is flagged and
+// replaced by 1 so that the step stays finite.
+__device__ __forceinline__ float pivot_rsqrt(float p, bool& bad) {
+  const bool ok = (p > 0.f) && (p < 3.0e38f);
+  bad |= !ok;
+  return rsqrt_nr(ok ? p : 1.f);
+}
+
+__device__ __forceinline__ void put4(float* dst, const float* v) {
 #pragma unroll
-    for (int r = 0; r < NB; ++r) v[r] = S[r * LDS + c];
-    colb[c] = S[c * LDS];         // column 0 (symmetric: row 0)
-  } else {
-    const int r = tid - NB;
+  for (int g = 0; g < HR / 4; ++g)
+    *reinterpret_cast<float4*>(dst + 4 * g) = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+}
+
+// v[i] -= sum_q c[q] X[q][i] for the thread's 32 entries; X: KB rows of stride NB
+__device__ __forceinline__ void rank4(float* v, const float* X, const float (&c)[KB]) {
 #pragma unroll
-    for (int c = 0; c < NB; ++c) v[c] = (c == r) ? 1.f : 0.f;
-    rowb[r] = (r == 0) ? 1.f : 0.f;
+  for (int g = 0; g < HR / 4; ++g) {
+    const float4 x0 = *reinterpret_cast<const float4*>(X + 0 * NB + 4 * g);
+    const float4 x1 = *reinterpret_cast<const float4*>(X + 1 * NB + 4 * g);
+    const float4 x2 = *reinterpret_cast<const float4*>(X + 2 * NB + 4 * g);
+    const float4 x3 = *reinterpret_cast<const float4*>(X + 3 * NB + 4 * g);
+    v[4 * g + 0] = fmaf(-c[0], x0.x, fmaf(-c[1], x1.x, fmaf(-c[2], x2.x, fmaf(-c[3], x3.x, v[4 * g + 0]))));
+    v[4 * g + 1] = fmaf(-c[0], x0.y, fmaf(-c[1], x1.y, fmaf(-c[2], x2.y, fmaf(-c[3], x3.y, v[4 * g + 1]))));
+    v[4 * g + 2] = fmaf(-c[0], x0.z, fmaf(-c[1], x1.z, fmaf(-c[2], x2.z, fmaf(-c[3], x3.z, v[4 * g + 2]))));
+    v[4 * g + 3] = fmaf(-c[0], x0.w, fmaf(-c[1], x1.w, fmaf(-c[2], x2.w, fmaf(-c[3], x3.w, v[4 * g + 3]))));
   }
+}
+
+// S: the block on entry, L on exit.  Ti: T on exit, and the broadcasts before.
+// Called by all GM_THREADS threads.
+__device__ __forceinline__ void block_factor(float* S, float* Ti, int32_t* st, const int tid) {
+  float* Pb = Ti;                        // [2][KB][NB]
+  float* Bb = Ti + 2 * KB * NB;          // [2][KB][NB]
+  float* cwb = Ti + 4 * KB * NB;         // [2][NB][KB]
+  const bool fac = tid < 2 * NB;
+  const int own = tid & (NB - 1);        // column (factor) or row (inverse) index
+  const int h = (tid >> 6) & 1;          // which half of it
+  float v[HR];
   bool bad = false;
-  df_bar();
-#pragma unroll 1
-  for (int j = 0; j <= NB; ++j) {
-    if (tid < NB) {
-      if (j < NB) {
-        const int c = tid;
-        const float* col = colb + (j & 1) * NB;
-        float p = col[j];
-        const bool okp = (p > 0.f) && (p < 3.0e38f);
-        bad |= (c == 0) && !okp;
-        p = okp ? p : 1.f;
-        const float inv = rsqrt_nr(p);
-        const float cc = col[c];
-        S[c * LDS + j] = (c > j) ? cc * inv : ((c == j) ? p * inv : 0.f);
-        if (c == 0) sinv[j] = inv;
-        if (c > j) {
-          const float sc = cc * inv * inv;
+  if (fac) {
 #pragma unroll
-          for (int q = 0; q < NB / 4; ++q) {
-            const float4 x = *reinterpret_cast<const float4*>(col + 4 * q);
-            v[4 * q + 0] = fmaf(-x.x, sc, v[4 * q + 0]);
-            v[4 * q + 1] = fmaf(-x.y, sc, v[4 * q + 1]);
-            v[4 * q + 2] = fmaf(-x.z, sc, v[4 * q + 2]);
-            v[4 * q + 3] = fmaf(-x.w, sc, v[4 * q + 3]);
-          }
-          if (c == j + 1) {
-            float* nx = colb + ((j + 1) & 1) * NB;
+    for (int i = 0; i < HR; ++i) v[i] = S[(HR * h + i) * LDS + own];
+  } else {
 #pragma unroll
-            for (int q = 0; q < NB / 4; ++q)
-              *reinterpret_cast<float4*>(nx + 4 * q) =
-                  make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-          }
-        }
-      }
-    } else if (j >= 1) {
-      // inverse step i = j - 1 (needs L[:, i] and 1/L[i][i], written in step i)
-      const int r = tid - NB, i = j - 1;
-      if (r > i) {
-        const float k = S[r * LDS + i] * sinv[i];
-        const float* row = rowb + (i & 1) * NB;
-#pragma unroll
-        for (int q = 0; q < NB / 4; ++q) {
-          const float4 x = *reinterpret_cast<const float4*>(row + 4 * q);
-          v[4 * q + 0] = fmaf(-k, x.x, v[4 * q + 0]);
-          v[4 * q + 1] = fmaf(-k, x.y, v[4 * q + 1]);
-          v[4 * q + 2] = fmaf(-k, x.z, v[4 * q + 2]);
-          v[4 * q + 3] = fmaf(-k, x.w, v[4 * q + 3]);
-        }
-        if (r == i + 1) {
-          float* nx = rowb + ((i + 1) & 1) * NB;
-#pragma unroll
-          for (int q = 0; q < NB / 4; ++q)
-            *reinterpret_cast<float4*>(nx + 4 * q) =
-                make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        }
-      }
-    }
-    df_bar();
+    for (int i = 0; i < HR; ++i) v[i] = (HR * h + i == own) ? 1.f : 0.f;
   }
-  if (tid >= NB) {
-    const int r = tid - NB;
-    const float ir = sinv[r];
+  __syncthreads();                       // S is read before the broadcasts start
+  if (own < KB) put4((fac ? Pb : Bb) + own * NB + HR * h, v);
+  __syncthreads();
+#pragma unroll 1
+  for (int b = 0; b <= NSTEP; ++b) {
+    if (fac) {
+      if (b < NSTEP) {
+        const int c = own, j0 = KB * b, cq = c - j0;
+        const float* P = Pb + (b & 1) * KB * NB;
+        // the pivot block (lower part) and the thread's own row of P
+        float a[KB][KB], pc[KB];
 #pragma unroll
-    for (int c = 0; c < NB; ++c) Ti[r * LDS + c] = (c <= r) ? v[c] * ir : 0.f;
+        for (int q = 0; q < KB; ++q) {
+          const float4 x = *reinterpret_cast<const float4*>(P + q * NB + j0);
+          a[0][q] = x.x; a[1][q] = x.y; a[2][q] = x.z; a[3][q] = x.w;   // a[row][col]
+          pc[q] = P[q * NB + c];
+        }
+        // L11 (lower) and its diagonal reciprocals
+        float l[KB][KB], id[KB];
+#pragma unroll
+        for (int q = 0; q < KB; ++q) {
+          float d = a[q][q];
+#pragma unroll
+          for (int k = 0; k < q; ++k) d = fmaf(-l[q][k], l[q][k], d);
+          id[q] = pivot_rsqrt(d, bad);
+          l[q][q] = d * id[q];
+#pragma unroll
+          for (int r = q + 1; r < KB; ++r) {
+            float x = a[r][q];
+#pragma unroll
+            for (int k = 0; k < q; ++k) x = fmaf(-l[r][k], l[q][k], x);
+            l[r][q] = x * id[q];
+          }
+        }
+        // M = L11^-1 (lower)
+        float m[KB][KB];
+#pragma unroll
+        for (int q = 0; q < KB; ++q) {
+          m[q][q] = id[q];
+#pragma unroll
+          for (int r = q + 1; r < KB; ++r) {
+            float x = 0.f;
+#pragma unroll
+            for (int k = q; k < r; ++k) x = fmaf(l[r][k], m[k][q], x);
+            m[r][q] = -x * id[r];
+          }
+        }
+        // own row of L: M p_c;  coefficients W p_c = M^T (M p_c)
+        float lr[KB], w[KB];
+#pragma unroll
+        for (int q = 0; q < KB; ++q) {
+          float x = 0.f;
+#pragma unroll
+          for (int k = 0; k <= q; ++k) x = fmaf(m[q][k], pc[k], x);
+          lr[q] = x;
+        }
+#pragma unroll
+        for (int q = 0; q < KB; ++q) {
+          float x = 0.f;
+#pragma unroll
+          for (int k = q; k < KB; ++k) x = fmaf(m[k][q], lr[k], x);
+          w[q] = x;
+        }
+        const bool below = cq >= KB, inblk = (cq >= 0) && !below;
+        if (h == 0) {
+          // coefficients for the inverse threads (row c of B), and L[c][j0..j0+3]
+          float cw[KB];
+#pragma unroll
+          for (int q = 0; q < KB; ++q) {
+            float mi = 0.f;
+#pragma unroll
+            for (int k = q; k < KB; ++k) mi = (cq == k) ? m[k][q] : mi;   // M is lower
+            cw[q] = below ? w[q] : (inblk ? ((cq == q ? 1.f : 0.f) - mi) : 0.f);
+          }
+          *reinterpret_cast<float4*>(cwb + (b & 1) * NB * KB + c * KB) =
+              make_float4(cw[0], cw[1], cw[2], cw[3]);
+#pragma unroll
+          for (int q = 0; q < KB; ++q)
+            S[c * LDS + j0 + q] = (below || (inblk && q <= cq)) ? lr[q] : 0.f;
+        }
+        // rank-4 update of the thread's column; columns at or left of the block
+        // take zero coefficients
+#pragma unroll
+        for (int q = 0; q < KB; ++q) w[q] = below ? w[q] : 0.f;
+        rank4(v, P + HR * h, w);
+        // the owners of the next block's columns publish them
+        if (cq >= KB && cq < 2 * KB) put4(Pb + ((b + 1) & 1) * KB * NB + (cq - KB) * NB + HR * h, v);
+      }
+    } else if (b >= 1) {
+      // inverse step for block b - 1
+      const int r = own, bb = b - 1, j0 = KB * bb, rq = r - j0;
+      const float4 cv = *reinterpret_cast<const float4*>(cwb + (bb & 1) * NB * KB + r * KB);
+      const float cw[KB] = {cv.x, cv.y, cv.z, cv.w};
+      rank4(v, Bb + (bb & 1) * KB * NB + HR * h, cw);
+      if (rq >= KB && rq < 2 * KB) put4(Bb + (b & 1) * KB * NB + (rq - KB) * NB + HR * h, v);
+    }
+    __syncthreads();
+  }
+  if (!fac) {
+#pragma unroll
+    for (int i = 0; i < HR; ++i) Ti[own * LDS + HR * h + i] = (HR * h + i <= own) ? v[i] : 0.f;
   }
   if (bad) raise_status(st, GPTQ_ERR_NOT_PD);
 }
@@ -266,7 +342,7 @@ __device__ __forceinline__ void diag_factor(float* A, int64_t lda, int k0, float
     S[(e >> 6) * LDS + (e & 63)] = A[int64_t(k0 + (e >> 6)) * lda + k0 + (e & 63)];
   }
   __syncthreads();
-  if (tid < 2 * NB) quad_factor(S, Ti, sm + DF_BCAST, st, tid);
+  block_factor(S, Ti, st, tid);
   __syncthreads();
 #pragma unroll
   for (int x = 0; x < (NB * NB) / GM_THREADS; ++x) {
