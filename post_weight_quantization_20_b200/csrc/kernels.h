@@ -24,11 +24,11 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
                          uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
                          float* losses, void* ws, int32_t* status);
 
-// trailing_tc.cu: W[:, e:] -= (Ehi + Elo) * U[i0:i0+128, e:] on tcgen05 (3xTF32),
-// with U given as its transposed split Ut_hi + Ut_lo (split_tf32_t)
+// trailing_tc.cu: W[:, e:cend] -= (Ehi + Elo) * U[i0:i0+128, e:cend] on tcgen05
+// (3xTF32), with U given as its transposed split Ut_hi + Ut_lo (split_tf32_t)
 bool trailing_tc_supported(int C);
 gptq_status split_tf32_t(cudaStream_t st, const float* U, int C, float* hi, float* lo);
-gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e,
+gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e, int cend,
                                const float* Ehi, const float* Elo, const float* Uthi,
                                const float* Utlo, int32_t* status);
 

@@ -413,6 +413,132 @@ __device__ __forceinline__ void lower_tile(int t, int& tm, int& tn) {
   tn = t - m * (m + 1) / 2;
 }
 
+// ---------------------------------------------------------------------------
+// The products of the factorization: 64x64 output tiles with K = 64, software
+// pipelined across a CTA's tiles.  A tile's operands (and its output, when the
+// tile accumulates into it) are fetched into registers while the CTA's previous
+// tile computes.  A is row-major (m, k); B is row-major (k, n) or stored (n, k);
+// an operand stored with k contiguous is read as float4 along k and transposed on
+// its way to shared memory (consecutive threads take consecutive rows, so the
+// stores hit distinct banks).  All extents are multiples of 64 and every tile
+// origin is 16-byte aligned (the factorization runs on a Cp x Cp copy, Cp a
+// multiple of 64).  A tile reads all of its operands before it writes, so its
+// output may overwrite an operand tile it alone reads (the in-place panel solve).
+// ---------------------------------------------------------------------------
+struct Tile64 {
+  const float* a;
+  const float* b;
+  float* d;
+  int64_t lda_, ldb, ldd;
+  float alpha;
+  bool bt;    // B stored (n, k)
+  bool acc;   // D += alpha A B (else D = alpha A B)
+};
+
+struct Fetch64 {
+  float4 a[4], b[4], d[4];
+};
+
+__device__ __forceinline__ float4 ld4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+
+__device__ __forceinline__ void fetch64(const Tile64& T, Fetch64& f) {
+  const int tid = threadIdx.x, rm = tid & 63, rq = tid >> 6;      // row, k-quad
+#pragma unroll
+  for (int i = 0; i < 4; ++i) f.a[i] = ld4(T.a + rm * T.lda_ + 4 * (rq + 4 * i));
+  if (T.bt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f.b[i] = ld4(T.b + rm * T.ldb + 4 * (rq + 4 * i));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f.b[i] = ld4(T.b + ((tid >> 4) + 16 * i) * T.ldb + 4 * (tid & 15));
+  }
+  if (T.acc) {
+    const int tx = tid & 15, ty = tid >> 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f.d[i] = ld4(T.d + (4 * ty + i) * T.ldd + 4 * tx);
+  }
+}
+
+// registers -> shared: As[k][m], Bs[k][n]
+__device__ __forceinline__ void stash64(bool bt, const Fetch64& f, float* sm) {
+  float* As = sm;
+  float* Bs = sm + GM_BK * GM_LD;
+  const int tid = threadIdx.x, rm = tid & 63, rq = tid >> 6;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int k = 4 * (rq + 4 * i);
+    As[(k + 0) * GM_LD + rm] = f.a[i].x;
+    As[(k + 1) * GM_LD + rm] = f.a[i].y;
+    As[(k + 2) * GM_LD + rm] = f.a[i].z;
+    As[(k + 3) * GM_LD + rm] = f.a[i].w;
+  }
+  if (bt) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int k = 4 * (rq + 4 * i);
+      Bs[(k + 0) * GM_LD + rm] = f.b[i].x;
+      Bs[(k + 1) * GM_LD + rm] = f.b[i].y;
+      Bs[(k + 2) * GM_LD + rm] = f.b[i].z;
+      Bs[(k + 3) * GM_LD + rm] = f.b[i].w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      *reinterpret_cast<float4*>(Bs + ((tid >> 4) + 16 * i) * GM_LD + 4 * (tid & 15)) = f.b[i];
+  }
+}
+
+// Runs work items t, t + step, ... < end; map(t) gives the item's tile.  Called
+// uniformly by the whole CTA; leaves sm free for reuse on return.
+template <class Map>
+__device__ __forceinline__ void run_tiles64(int t, int step, int end, const Map& map, float* sm) {
+  if (t >= end) return;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  Tile64 T = map(t);
+  Fetch64 f;
+  fetch64(T, f);
+  for (;;) {
+    __syncthreads();                       // the previous tile is done with sm
+    stash64(T.bt, f, sm);
+    float4 dold[4] = {f.d[0], f.d[1], f.d[2], f.d[3]};
+    float* const d = T.d;
+    const int64_t ldd = T.ldd;
+    const float alpha = T.alpha;
+    const bool acc = T.acc;
+    __syncthreads();
+    const int tnext = t + step;
+    if (tnext < end) {
+      T = map(tnext);
+      fetch64(T, f);
+    }
+    const float* As = sm;
+    const float* Bs = sm + GM_BK * GM_LD;
+    float c[4][4] = {};
+#pragma unroll 16
+    for (int kk = 0; kk < GM_BK; ++kk) {
+      const float4 x = *reinterpret_cast<const float4*>(As + kk * GM_LD + 4 * ty);
+      const float4 y = *reinterpret_cast<const float4*>(Bs + kk * GM_LD + 4 * tx);
+      const float xv[4] = {x.x, x.y, x.z, x.w};
+      const float yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) c[i][j] = fmaf(xv[i], yv[j], c[i][j]);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float4 o = make_float4(alpha * c[i][0], alpha * c[i][1], alpha * c[i][2], alpha * c[i][3]);
+      if (acc) {
+        o.x += dold[i].x; o.y += dold[i].y; o.z += dold[i].z; o.w += dold[i].w;
+      }
+      *reinterpret_cast<float4*>(d + (4 * ty + i) * ldd + 4 * tx) = o;
+    }
+    if (tnext >= end) break;
+    t = tnext;
+  }
+  __syncthreads();
+}
+
 __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs a) {
   // one buffer: GEMM chunks, or the tiles of the diagonal factor
   __shared__ __align__(16) float sm[GM_SMEM_FLOATS];
@@ -427,41 +553,61 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
     const int nr = rest / NB;
     float* panel = a.A + int64_t(k0 + NB) * lda + k0;
     float* brow = a.Bx + int64_t(k0) * lda;
-    // phase A
-    const GemmProb pan = make_prob(rest, NB, NB, 1.f, panel, lda, 1, Tk, 1, NB, 0.f, panel, lda, 0);
-    const GemmProb xk = make_prob(NB, k0 + NB, NB, 1.f, Tk, NB, 1, brow, lda, 1, 0.f, brow, lda, 0);
-    for (int t = blockIdx.x; t < pan.ntiles + xk.ntiles; t += gridDim.x) {
-      if (t < pan.ntiles) gemm_tile(pan, t, 0, sm);
-      else gemm_tile(xk, 0, t - pan.ntiles, sm);
-    }
+    // phase A: the panel solve L[k0+64:, k] = A[k0+64:, k] T_k^T (in place), and
+    // X_k = T_k Bx[k, 0:k0+64] (in place)
+    const auto phase_a = [&](int t) {
+      Tile64 T;
+      if (t < nr) {
+        T.a = panel + int64_t(t) * NB * lda; T.lda_ = lda;
+        T.b = Tk;                            T.ldb = NB;  T.bt = true;
+        T.d = panel + int64_t(t) * NB * lda; T.ldd = lda;
+      } else {
+        const int u = t - nr;
+        T.a = Tk;                            T.lda_ = NB;
+        T.b = brow + u * NB;                 T.ldb = lda; T.bt = false;
+        T.d = brow + u * NB;                 T.ldd = lda;
+      }
+      T.alpha = 1.f;
+      T.acc = false;
+      return T;
+    };
+    run_tiles64(blockIdx.x, gridDim.x, nr + k + 1, phase_a, sm);
     if (!grid_barrier(a, epoch)) return;
     if (rest == 0) break;
-    // phase B
-    const GemmProb syrk = make_prob(rest, rest, NB, -1.f, panel, lda, 1, panel, 1, lda, 1.f,
-                                    a.A + int64_t(k0 + NB) * lda + k0 + NB, lda, 1);
-    const GemmProb bup = make_prob(rest, k0 + NB, NB, -1.f, panel, lda, 1, brow, lda, 1, 1.f,
-                                   a.Bx + int64_t(k0 + NB) * lda, lda, 0);
+    // phase B: A[k0+64:, k0+64:] -= P P^T (lower tiles) and
+    // Bx[k0+64:, 0:k0+64] -= P X_k
     const int n_syrk = nr * (nr + 1) / 2;
-    const int n_total = n_syrk + bup.ntiles;
+    const int n_total = n_syrk + nr * (k + 1);
+    float* trail = a.A + int64_t(k0 + NB) * lda + k0 + NB;
+    float* bxb = a.Bx + int64_t(k0 + NB) * lda;
+    const auto phase_b = [&](int t) {
+      Tile64 T;
+      int tm, tn;
+      if (t < n_syrk) {
+        lower_tile(t, tm, tn);
+        T.b = panel + int64_t(tn) * NB * lda; T.ldb = lda; T.bt = true;
+        T.d = trail + int64_t(tm) * NB * lda + tn * NB;
+      } else {
+        const int u = t - n_syrk;
+        tm = u / (k + 1);
+        tn = u - tm * (k + 1);
+        T.b = brow + tn * NB;                 T.ldb = lda; T.bt = false;
+        T.d = bxb + int64_t(tm) * NB * lda + tn * NB;
+      }
+      T.a = panel + int64_t(tm) * NB * lda;
+      T.lda_ = lda;
+      T.ldd = lda;
+      T.alpha = -1.f;
+      T.acc = true;
+      return T;
+    };
     if (blockIdx.x == 0) {
-      gemm_tile(syrk, 0, 0, sm);
-      __syncthreads();
+      run_tiles64(0, 1, 1, phase_b, sm);     // the next diagonal block first
       diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, sm);
     }
     const int workers = gridDim.x > 1 ? gridDim.x - 1 : 1;
     const int first = gridDim.x > 1 ? int(blockIdx.x) - 1 : 0;
-    if (gridDim.x == 1 || blockIdx.x > 0) {
-      for (int t = 1 + first; t < n_total; t += workers) {
-        if (t < n_syrk) {
-          int tm, tn;
-          lower_tile(t, tm, tn);
-          gemm_tile(syrk, tm, tn, sm);
-        } else {
-          const int u = t - n_syrk;
-          gemm_tile(bup, u / bup.tiles_n, u % bup.tiles_n, sm);
-        }
-      }
-    }
+    if (gridDim.x == 1 || blockIdx.x > 0) run_tiles64(1 + first, workers, n_total, phase_b, sm);
     if (!grid_barrier(a, epoch)) return;
   }
 }

@@ -3,7 +3,8 @@
 //
 // Data layout in HBM (workspace):
 //   Wk    rows x C fp32   working copy of W in sweep order (columns gathered by perm)
-//   Err   rows x 128 fp32 scaled errors (w - Q)/U[q][q] of the current panel
+//   Err   2 x rows x 128 fp32 scaled errors (w - Q)/U[q][q] of a panel, split hi + lo,
+//         double-buffered by panel parity
 //   cp    rows x C u8     codes in sweep order
 //   lpart tiles x C fp32  per-row-tile partial column losses (summed in finalize)
 //
@@ -33,8 +34,8 @@ constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_ROWS * SW_B) * 4;
 
 struct QuantLayout {
   float* Wk;
-  float* Ehi;
-  float* Elo;
+  float* Ehi[2];
+  float* Elo[2];
   uint8_t* cp;
   float* lpart;
   float* Uhi;
@@ -47,8 +48,10 @@ static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
   L.tiles = int((R + SW_ROWS - 1) / SW_ROWS);
   char* p = static_cast<char*>(ws);
   L.Wk = reinterpret_cast<float*>(p);    p += align256(size_t(R) * C * 4);
-  L.Ehi = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_B * 4);
-  L.Elo = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_B * 4);
+  for (int b = 0; b < 2; ++b) {
+    L.Ehi[b] = reinterpret_cast<float*>(p); p += align256(size_t(R) * SW_B * 4);
+    L.Elo[b] = reinterpret_cast<float*>(p); p += align256(size_t(R) * SW_B * 4);
+  }
   L.cp = reinterpret_cast<uint8_t*>(p);  p += align256(size_t(R) * C);
   L.lpart = reinterpret_cast<float*>(p); p += align256(size_t(L.tiles) * C * 4);
   L.Uhi = reinterpret_cast<float*>(p);   p += align256(size_t(C) * C * 4);
@@ -58,7 +61,7 @@ static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
 
 size_t quantize_ws_bytes(int64_t R, int64_t C, const gptq_config&) {
   const int64_t tiles = (R + SW_ROWS - 1) / SW_ROWS;
-  return align256(size_t(R) * C * 4) + 2 * align256(size_t(R) * SW_B * 4) +
+  return align256(size_t(R) * C * 4) + 4 * align256(size_t(R) * SW_B * 4) +
          align256(size_t(R) * C) + align256(size_t(tiles) * C * 4) +
          2 * align256(size_t(C) * C * 4) + 256;
 }
@@ -290,6 +293,101 @@ __global__ void k_finalize_cols(const float* lpart, int tiles, int C, const int3
 
 static int grid_for(int64_t n) { return int(std::min<int64_t>((n + 255) / 256, 148 * 32)); }
 
+// One non-blocking side stream per host thread and device, created on first use.
+static cudaStream_t side_stream(gptq_status& err) {
+  static thread_local cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64) {
+    note_error(e == cudaSuccess ? cudaErrorInvalidDevice : e, "side_stream");
+    err = GPTQ_ERR_CUDA;
+    return nullptr;
+  }
+  if (!streams[dev]) {
+    e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) {
+      note_error(e, "cudaStreamCreateWithFlags");
+      streams[dev] = nullptr;
+      err = GPTQ_ERR_CUDA;
+      return nullptr;
+    }
+  }
+  err = GPTQ_OK;
+  return streams[dev];
+}
+
+// The panels with the lazy trailing update split in two (a lookahead of one
+// panel): after the sweep of panel p, the caller's stream updates only the next
+// panel's columns and goes on to sweep it, while a side stream applies panel p's
+// update to all later columns.  Order: the side update of panel p starts after
+// the sweep of p; the next-panel update of p+1 touches columns the side update
+// of p also writes, so it waits for it.  Panel errors are double-buffered, and
+// the sweep of p+2 (which overwrites p's buffer) comes after the next-panel
+// update of p+1, hence after the side update of p.  The caller's stream joins
+// the side stream before returning, so work enqueued after this call, and a
+// stream capture of it, sees the whole update.
+static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R, int C,
+                                   const float* U, const gptq_config& cfg, int g, int G,
+                                   float* scales, float* zeros, int32_t* status) {
+  gptq_status err = GPTQ_OK;
+  cudaStream_t side = side_stream(err);
+  if (err != GPTQ_OK) return err;
+  cudaEvent_t swept = nullptr, updated = nullptr;
+  GPTQ_CUDA(cudaEventCreateWithFlags(&swept, cudaEventDisableTiming));
+  cudaError_t ce = cudaEventCreateWithFlags(&updated, cudaEventDisableTiming);
+  if (ce != cudaSuccess) {
+    cudaEventDestroy(swept);
+    note_error(ce, "cudaEventCreateWithFlags");
+    return GPTQ_ERR_CUDA;
+  }
+  // fork: the side stream starts after everything the caller enqueued so far
+  ce = cudaEventRecord(swept, st);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
+  bool pending = false;   // a side update has been enqueued since the last join
+  for (int i0 = 0; i0 < C && ce == cudaSuccess && err == GPTQ_OK; i0 += SW_B) {
+    const int p = (i0 / SW_B) & 1;
+    const int nb = min(SW_B, C - i0);
+    k_sweep_panel<<<L.tiles, SW_THREADS, SW_SMEM, st>>>(L.Wk, R, C, i0, nb, U, cfg.bits, g,
+                                                        cfg.sym, scales, zeros, G, L.cp,
+                                                        L.Ehi[p], L.Elo[p], L.lpart);
+    note_launch();
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) break;
+    const int e = i0 + nb;
+    if (e >= C) break;
+    const int nx = min(e + SW_B, C);
+    if (nx < C) {
+      ce = cudaEventRecord(swept, st);
+      if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
+      if (ce != cudaSuccess) break;
+    }
+    if (pending) {
+      ce = cudaStreamWaitEvent(st, updated, 0);
+      if (ce != cudaSuccess) break;
+      pending = false;
+    }
+    err = trailing_update_tc(st, L.Wk, R, C, i0, e, nx, L.Ehi[p], L.Elo[p], L.Uhi, L.Ulo, status);
+    if (err == GPTQ_OK && nx < C) {
+      err = trailing_update_tc(side, L.Wk, R, C, i0, nx, C, L.Ehi[p], L.Elo[p], L.Uhi, L.Ulo,
+                               status);
+      if (err == GPTQ_OK) {
+        ce = cudaEventRecord(updated, side);
+        pending = true;
+      }
+    }
+  }
+  // join (also after an error, so that nothing is left running on the side stream
+  // unordered with the caller's stream)
+  if (cudaEventRecord(updated, side) == cudaSuccess) cudaStreamWaitEvent(st, updated, 0);
+  cudaEventDestroy(swept);
+  cudaEventDestroy(updated);
+  if (ce != cudaSuccess) {
+    note_error(ce, "sweep_lookahead");
+    return GPTQ_ERR_CUDA;
+  }
+  return err;
+}
+
 gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, int64_t ldw,
                          const float* U, const int32_t* perm, const gptq_config& cfg,
                          uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
@@ -307,21 +405,21 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
     GPTQ_LAUNCH(k_row_grid, (R + 7) / 8, 256, 0, st, L.Wk, R, C, cfg.bits, cfg.sym, scales, zeros);
   }
   const bool tc = C > SW_B && trailing_tc_supported(C);
-  if (tc) GPTQ_TRY(split_tf32_t(st, U, C, L.Uhi, L.Ulo));
-  for (int i0 = 0; i0 < C; i0 += SW_B) {
-    const int nb = min(SW_B, C - i0);
-    GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
-                g, cfg.sym, scales, zeros, G, L.cp, L.Ehi, L.Elo, L.lpart);
-    const int e = i0 + nb;
-    if (e < C) {
-      // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]
-      if (tc) {
-        GPTQ_TRY(trailing_update_tc(st, L.Wk, R, C, i0, e, L.Ehi, L.Elo, L.Uhi, L.Ulo, status));
-      } else {
-        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Ehi, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
-                          1.f, L.Wk + e, C, 0));
-        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Elo, SW_B, 1, U + int64_t(i0) * C + e, C, 1,
-                          1.f, L.Wk + e, C, 0));
+  if (tc) {
+    GPTQ_TRY(split_tf32_t(st, U, C, L.Uhi, L.Ulo));
+    GPTQ_TRY(sweep_lookahead(st, L, R, C, U, cfg, g, G, scales, zeros, status));
+  } else {
+    for (int i0 = 0; i0 < C; i0 += SW_B) {
+      const int nb = min(SW_B, C - i0);
+      GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
+                  g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[0], L.Elo[0], L.lpart);
+      const int e = i0 + nb;
+      if (e < C) {
+        // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Ehi[0], SW_B, 1, U + int64_t(i0) * C + e, C,
+                          1, 1.f, L.Wk + e, C, 0));
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Elo[0], SW_B, 1, U + int64_t(i0) * C + e, C,
+                          1, 1.f, L.Wk + e, C, 0));
       }
     }
   }

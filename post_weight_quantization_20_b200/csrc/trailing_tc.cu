@@ -1,6 +1,8 @@
 // Lazy trailing update on the tensor cores, GPTQ量化算法深度解析 §2.4:
-//   W[:, e:] -= Err * U[i0:e, e:]
-// Err (rows x 128) holds the scaled errors of the panel just swept.  The product
+//   W[:, e:cend] -= Err * U[i0:e, e:cend]
+// Err (rows x 128) holds the scaled errors of the panel just swept; a call may
+// cover any column range after the panel (the sweep updates the next panel's
+// columns first and the rest concurrently).  The product
 // is fp32-faithful by a 3xTF32 split: x = hi + lo with hi = x with its low 13
 // mantissa bits cleared (exact in tf32) and lo = x - hi, and
 //   Err * U ~= Err_hi U_hi + Err_hi U_lo + Err_lo U_hi
@@ -32,7 +34,8 @@ constexpr int SMEM = BUFS * STAGE + 1024 + 128;
 __global__ void __launch_bounds__(THREADS, 1)
 k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ CUtensorMap elo,
               const __grid_constant__ CUtensorMap uhi, const __grid_constant__ CUtensorMap ulo,
-              float* Wk, int R, int C, int i0, int e, uint32_t idesc, int vec, int32_t* status) {
+              float* Wk, int R, int C, int i0, int e, int cend, uint32_t idesc, int vec,
+              int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -120,7 +123,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
       tc::tmem_ld_wait();
       const int col = n0 + c * 16;
       if (!rv) continue;
-      if (vec && col + 16 <= C) {
+      if (vec && col + 16 <= cend) {
         float4* p = reinterpret_cast<float4*>(wrow + col);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -134,7 +137,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
       } else {
 #pragma unroll
         for (int q = 0; q < 16; ++q)
-          if (col + q < C) wrow[col + q] -= __uint_as_float(v[q]);
+          if (col + q < cend) wrow[col + q] -= __uint_as_float(v[q]);
       }
     }
   }
@@ -202,10 +205,10 @@ gptq_status split_tf32_t(cudaStream_t st, const float* U, int C, float* hi, floa
   return GPTQ_OK;
 }
 
-gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e,
+gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e, int cend,
                                const float* Ehi, const float* Elo, const float* Uthi,
                                const float* Utlo, int32_t* status) {
-  if (e >= C || R <= 0) return GPTQ_OK;
+  if (e >= cend || cend > C || R <= 0) return GPTQ_OK;
   CUtensorMap mehi, melo, muhi, mulo;
   if (!encode_2d(&mehi, Ehi, 128, uint64_t(R), 128, TK, TM) ||
       !encode_2d(&melo, Elo, 128, uint64_t(R), 128, TK, TM) ||
@@ -217,9 +220,9 @@ gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0,
                          (uint32_t(TM >> 4) << 24);
   const int vec = ((C & 3) == 0 && (reinterpret_cast<uintptr_t>(Wk) & 15) == 0) ? 1 : 0;
   GPTQ_CUDA(allow_smem(k_trailing_tc, SMEM));
-  dim3 grid((C - e + TN - 1) / TN, (R + TM - 1) / TM);
+  dim3 grid((cend - e + TN - 1) / TN, (R + TM - 1) / TM);
   GPTQ_LAUNCH(k_trailing_tc, grid, THREADS, SMEM, st, mehi, melo, muhi, mulo, Wk, R, C, i0, e,
-              idesc, vec, status);
+              cend, idesc, vec, status);
   return GPTQ_OK;
 }
 
