@@ -29,8 +29,9 @@ constexpr int SW_CPT = SW_B / SW_TPR;     // panel columns owned by one thread (
 constexpr int SW_ROWS = 16;               // rows per CTA
 constexpr int SW_THREADS = SW_ROWS * SW_TPR;
 constexpr int SW_LDU = SW_B + 4 * SW_TPR; // skewed U row: column c at c + 4*(c / SW_CPT)
-// U block, 1/U_qq, per-row losses of the panel
-constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_ROWS * SW_B) * 4;
+constexpr int SW_LDE = SW_B + 1;           // staged error row (the previous panel's)
+// U block, 1/U_qq, per-row losses of the panel (or the previous panel's errors)
+constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_ROWS * SW_LDE) * 4;
 
 struct QuantLayout {
   float* Wk;
@@ -124,32 +125,45 @@ __device__ __forceinline__ int uskew(int b) { return b + 4 * (b / SW_CPT); }
 __global__ void __launch_bounds__(SW_THREADS)
 k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits, int g, int sym,
               float* scales, float* zeros, int G, uint8_t* cp, float* Ehi, float* Elo,
-              float* lpart) {
+              float* lpart, const float* Eph, const float* Epl, int ip) {
   extern __shared__ __align__(16) float sm[];
   float* Us = sm;                       // SW_B x SW_LDU
   float* dinv = Us + SW_B * SW_LDU;     // SW_B
-  float* lrow = dinv + SW_B;            // SW_ROWS x SW_B
+  float* lrow = dinv + SW_B;            // SW_ROWS x SW_LDE
   const int tid = threadIdx.x, lane = tid & 31;
   const int t = tid % SW_TPR, rl = tid / SW_TPR;
   const int r = blockIdx.x * SW_ROWS + rl;
   const bool rv = r < R;
-  // U block (rows and columns i0 .. i0 + nb) into the skewed layout, 16-byte loads
   const bool vec = ((C & 3) == 0) && (nb == SW_B) && ((reinterpret_cast<uintptr_t>(U) & 15) == 0);
-  if (vec) {
-#pragma unroll 8
-    for (int x = 0; x < (SW_B * SW_B / 4) / SW_THREADS; ++x) {
-      const int e4 = tid + SW_THREADS * x;
-      const int a = e4 / (SW_B / 4), b = 4 * (e4 % (SW_B / 4));
-      const float4 v = *reinterpret_cast<const float4*>(U + int64_t(i0 + a) * C + i0 + b);
-      *reinterpret_cast<float4*>(Us + a * SW_LDU + uskew(b)) = v;
+  // U[a0 .. a0+128, i0 .. i0+nb) into the skewed layout, 16-byte loads
+  const auto load_ublock = [&](int a0, int na) {
+    if (vec) {
+      // batches of 16 loads issued before their stores (a generic-pointer load
+      // may not move past a shared store the compiler cannot tell apart from it)
+      constexpr int NX = (SW_B * SW_B / 4) / SW_THREADS, BX = 16;
+#pragma unroll 1
+      for (int x0 = 0; x0 < NX; x0 += BX) {
+        float4 v[BX];
+#pragma unroll
+        for (int x = 0; x < BX; ++x) {
+          const int e4 = tid + SW_THREADS * (x0 + x);
+          const int a = e4 / (SW_B / 4), b = 4 * (e4 % (SW_B / 4));
+          v[x] = *reinterpret_cast<const float4*>(U + int64_t(a0 + a) * C + i0 + b);
+        }
+#pragma unroll
+        for (int x = 0; x < BX; ++x) {
+          const int e4 = tid + SW_THREADS * (x0 + x);
+          const int a = e4 / (SW_B / 4), b = 4 * (e4 % (SW_B / 4));
+          *reinterpret_cast<float4*>(Us + a * SW_LDU + uskew(b)) = v[x];
+        }
+      }
+    } else {
+      for (int e = tid; e < SW_B * SW_B; e += SW_THREADS) {
+        const int a = e / SW_B, b = e % SW_B;
+        Us[a * SW_LDU + uskew(b)] = (a < na && b < nb) ? U[int64_t(a0 + a) * C + i0 + b] : 0.f;
+      }
     }
-  } else {
-    for (int e = tid; e < SW_B * SW_B; e += SW_THREADS) {
-      const int a = e / SW_B, b = e % SW_B;
-      Us[a * SW_LDU + uskew(b)] = (a < nb && b < nb) ? U[int64_t(i0 + a) * C + i0 + b] : 0.f;
-    }
-  }
-  if (tid < SW_B) dinv[tid] = tid < nb ? 1.f / U[int64_t(i0 + tid) * C + i0 + tid] : 0.f;
+  };
   float w[SW_CPT];
   const float* wrow = Wk + int64_t(rv ? r : 0) * C + i0 + t * SW_CPT;
   if (rv && vec) {
@@ -162,6 +176,52 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
 #pragma unroll
     for (int jj = 0; jj < SW_CPT; ++jj) w[jj] = (rv && t * SW_CPT + jj < nb) ? wrow[jj] : 0.f;
   }
+  if (ip >= 0) {
+    // the previous panel's lazy update restricted to this panel's columns, in fp32:
+    // W[:, i0:i0+nb] -= Err_prev * U[ip:ip+128, i0:i0+nb]
+    {
+      // the CTA's rows of the previous errors: all loads in flight at once
+      constexpr int NQ = SW_ROWS * SW_B / 4 / SW_THREADS;
+      float4 hq[NQ], lq[NQ];
+#pragma unroll
+      for (int x = 0; x < NQ; ++x) {
+        const int e4 = tid + SW_THREADS * x, rr = e4 / (SW_B / 4), k = 4 * (e4 % (SW_B / 4));
+        const int row = blockIdx.x * SW_ROWS + rr;
+        const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        hq[x] = row < R ? *reinterpret_cast<const float4*>(Eph + int64_t(row) * SW_B + k) : zero4;
+        lq[x] = row < R ? *reinterpret_cast<const float4*>(Epl + int64_t(row) * SW_B + k) : zero4;
+      }
+      load_ublock(ip, SW_B);
+#pragma unroll
+      for (int x = 0; x < NQ; ++x) {
+        const int e4 = tid + SW_THREADS * x, rr = e4 / (SW_B / 4), k = 4 * (e4 % (SW_B / 4));
+        float* d = lrow + rr * SW_LDE + k;
+        d[0] = hq[x].x + lq[x].x;
+        d[1] = hq[x].y + lq[x].y;
+        d[2] = hq[x].z + lq[x].z;
+        d[3] = hq[x].w + lq[x].w;
+      }
+    }
+    __syncthreads();
+    const float* erow = lrow + rl * SW_LDE;
+#pragma unroll 4
+    for (int k = 0; k < SW_B; ++k) {
+      const float ek = erow[k];
+      const float* urow = Us + k * SW_LDU + t * (SW_CPT + 4);
+#pragma unroll
+      for (int jj = 0; jj < SW_CPT; jj += 4) {
+        const float4 u = *reinterpret_cast<const float4*>(urow + jj);
+        w[jj + 0] = fmaf(-ek, u.x, w[jj + 0]);
+        w[jj + 1] = fmaf(-ek, u.y, w[jj + 1]);
+        w[jj + 2] = fmaf(-ek, u.z, w[jj + 2]);
+        w[jj + 3] = fmaf(-ek, u.w, w[jj + 3]);
+      }
+    }
+    __syncthreads();   // Us and lrow are reused below
+  }
+  // the panel's own U block (rows and columns i0 .. i0 + nb)
+  load_ublock(i0, nb);
+  if (tid < SW_B) dinv[tid] = tid < nb ? 1.f / U[int64_t(i0 + tid) * C + i0 + tid] : 0.f;
   __syncthreads();
 
   const float maxq = float((1 << bits) - 1);
@@ -255,12 +315,12 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
     }
   }
 #pragma unroll
-  for (int jj = 0; jj < SW_CPT; ++jj) lrow[rl * SW_B + t * SW_CPT + jj] = rv ? 0.5f * e[jj] * e[jj] : 0.f;
+  for (int jj = 0; jj < SW_CPT; ++jj) lrow[rl * SW_LDE + t * SW_CPT + jj] = rv ? 0.5f * e[jj] * e[jj] : 0.f;
   __syncthreads();
   if (tid < nb) {
     float l = 0.f;
 #pragma unroll
-    for (int i = 0; i < SW_ROWS; ++i) l += lrow[i * SW_B + tid];
+    for (int i = 0; i < SW_ROWS; ++i) l += lrow[i * SW_LDE + tid];
     lpart[int64_t(blockIdx.x) * C + i0 + tid] = l;
   }
 }
@@ -317,70 +377,67 @@ static cudaStream_t side_stream(gptq_status& err) {
 }
 
 // The panels with the lazy trailing update split in two (a lookahead of one
-// panel): after the sweep of panel p, the caller's stream updates only the next
-// panel's columns and goes on to sweep it, while a side stream applies panel p's
-// update to all later columns.  Order: the side update of panel p starts after
-// the sweep of p; the next-panel update of p+1 touches columns the side update
-// of p also writes, so it waits for it.  Panel errors are double-buffered, and
-// the sweep of p+2 (which overwrites p's buffer) comes after the next-panel
-// update of p+1, hence after the side update of p.  The caller's stream joins
-// the side stream before returning, so work enqueued after this call, and a
-// stream capture of it, sees the whole update.
+// panel).  The sweep of panel p first applies panel p-1's update to its own
+// columns (in fp32, from the errors p-1 left in its buffer), then sweeps; a side
+// stream applies panel p's update to the columns from panel p+2 on.  Order: the
+// side update of p starts after the sweep of p; the sweep of p waits for the side
+// update of p-2, the last one that writes its columns (side updates run in panel
+// order on the side stream).  Panel errors alternate between two buffers, and the
+// sweep of p+2, which overwrites p's, waits for the side update of p, the last
+// reader.  The caller's stream joins the side stream before returning (event
+// fork/join, so the call can be stream-captured).  Every column receives its
+// panel updates in panel order, so results are deterministic.
 static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R, int C,
                                    const float* U, const gptq_config& cfg, int g, int G,
                                    float* scales, float* zeros, int32_t* status) {
   gptq_status err = GPTQ_OK;
   cudaStream_t side = side_stream(err);
   if (err != GPTQ_OK) return err;
-  cudaEvent_t swept = nullptr, updated = nullptr;
-  GPTQ_CUDA(cudaEventCreateWithFlags(&swept, cudaEventDisableTiming));
-  cudaError_t ce = cudaEventCreateWithFlags(&updated, cudaEventDisableTiming);
+  cudaEvent_t ev[3] = {};   // swept, updated[2]
+  cudaError_t ce = cudaSuccess;
+  for (int i = 0; i < 3 && ce == cudaSuccess; ++i)
+    ce = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming);
   if (ce != cudaSuccess) {
-    cudaEventDestroy(swept);
+    for (cudaEvent_t e : ev)
+      if (e) cudaEventDestroy(e);
     note_error(ce, "cudaEventCreateWithFlags");
     return GPTQ_ERR_CUDA;
   }
+  cudaEvent_t swept = ev[0];
   // fork: the side stream starts after everything the caller enqueued so far
   ce = cudaEventRecord(swept, st);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
-  bool pending = false;   // a side update has been enqueued since the last join
-  for (int i0 = 0; i0 < C && ce == cudaSuccess && err == GPTQ_OK; i0 += SW_B) {
-    const int p = (i0 / SW_B) & 1;
-    const int nb = min(SW_B, C - i0);
-    k_sweep_panel<<<L.tiles, SW_THREADS, SW_SMEM, st>>>(L.Wk, R, C, i0, nb, U, cfg.bits, g,
-                                                        cfg.sym, scales, zeros, G, L.cp,
-                                                        L.Ehi[p], L.Elo[p], L.lpart);
+  bool upd[2] = {false, false};   // updated[b] holds the side update of an earlier panel
+  const int np = (C + SW_B - 1) / SW_B;
+  for (int p = 0; p < np && ce == cudaSuccess && err == GPTQ_OK; ++p) {
+    const int i0 = p * SW_B, nb = min(SW_B, C - i0), b = p & 1;
+    if (upd[b]) {   // the side update of p-2
+      ce = cudaStreamWaitEvent(st, ev[1 + b], 0);
+      if (ce != cudaSuccess) break;
+      upd[b] = false;
+    }
+    const int pb = (p - 1) & 1;
+    k_sweep_panel<<<L.tiles, SW_THREADS, SW_SMEM, st>>>(
+        L.Wk, R, C, i0, nb, U, cfg.bits, g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[b], L.Elo[b],
+        L.lpart, L.Ehi[pb], L.Elo[pb], p > 0 ? i0 - SW_B : -1);
     note_launch();
     ce = cudaGetLastError();
     if (ce != cudaSuccess) break;
-    const int e = i0 + nb;
-    if (e >= C) break;
-    const int nx = min(e + SW_B, C);
-    if (nx < C) {
-      ce = cudaEventRecord(swept, st);
-      if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
-      if (ce != cudaSuccess) break;
-    }
-    if (pending) {
-      ce = cudaStreamWaitEvent(st, updated, 0);
-      if (ce != cudaSuccess) break;
-      pending = false;
-    }
-    err = trailing_update_tc(st, L.Wk, R, C, i0, e, nx, L.Ehi[p], L.Elo[p], L.Uhi, L.Ulo, status);
-    if (err == GPTQ_OK && nx < C) {
-      err = trailing_update_tc(side, L.Wk, R, C, i0, nx, C, L.Ehi[p], L.Elo[p], L.Uhi, L.Ulo,
-                               status);
-      if (err == GPTQ_OK) {
-        ce = cudaEventRecord(updated, side);
-        pending = true;
-      }
-    }
+    const int e = i0 + nb + SW_B;   // the side update covers columns from panel p+2 on
+    if (e >= C) continue;
+    ce = cudaEventRecord(swept, st);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
+    if (ce != cudaSuccess) break;
+    err = trailing_update_tc(side, L.Wk, R, C, i0, e, C, L.Ehi[b], L.Elo[b], L.Uhi, L.Ulo,
+                             status);
+    if (err != GPTQ_OK) break;
+    ce = cudaEventRecord(ev[1 + b], side);
+    upd[b] = ce == cudaSuccess;
   }
   // join (also after an error, so that nothing is left running on the side stream
   // unordered with the caller's stream)
-  if (cudaEventRecord(updated, side) == cudaSuccess) cudaStreamWaitEvent(st, updated, 0);
-  cudaEventDestroy(swept);
-  cudaEventDestroy(updated);
+  if (cudaEventRecord(swept, side) == cudaSuccess) cudaStreamWaitEvent(st, swept, 0);
+  for (cudaEvent_t e : ev) cudaEventDestroy(e);
   if (ce != cudaSuccess) {
     note_error(ce, "sweep_lookahead");
     return GPTQ_ERR_CUDA;
@@ -412,7 +469,8 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
     for (int i0 = 0; i0 < C; i0 += SW_B) {
       const int nb = min(SW_B, C - i0);
       GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
-                  g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[0], L.Elo[0], L.lpart);
+                  g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[0], L.Elo[0], L.lpart, nullptr,
+                  nullptr, -1);
       const int e = i0 + nb;
       if (e < C) {
         // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]

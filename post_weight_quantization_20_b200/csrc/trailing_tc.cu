@@ -14,7 +14,8 @@
 // in flight (96 KB each: Err hi+lo and Ut hi+lo K-major boxes of 32 K-values x
 // 128 rows, 128-byte swizzled by TMA).  Warp 0 issues TMA, warp 1 issues tcgen05.mma
 // kind::tf32 (M=128, N=256, K=8) into one 256-column TMEM accumulator, then all
-// four warps read the accumulator and subtract it from the fp32 working copy.
+// four warps move the accumulator through shared memory and subtract it from the
+// fp32 working copy in coalesced row segments.
 #include <algorithm>
 
 #include "kernels.h"
@@ -30,6 +31,8 @@ constexpr int STAGE = 2 * A_BOX + 2 * (TN / 128) * B_BOX;  // 96 KB
 constexpr int BUFS = 2;
 constexpr int THREADS = 128;
 constexpr int SMEM = BUFS * STAGE + 1024 + 128;
+constexpr int EP_LD = TN + 4;                              // staged accumulator row (floats)
+static_assert(TM * EP_LD * 4 <= BUFS * STAGE, "the stage buffers hold the accumulator tile");
 
 __global__ void __launch_bounds__(THREADS, 1)
 k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ CUtensorMap elo,
@@ -109,35 +112,67 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
     }
     if (ok) tc::mma_commit(done);
   }
-  // epilogue: all four warps; warp w owns TMEM lanes (rows) 32w .. 32w + 31
+  // epilogue: the accumulator goes through shared memory (the stage buffers are
+  // free once every MMA has completed) so that W is updated with coalesced row
+  // segments and many loads in flight.  Warp w owns TMEM lanes (rows) 32w..32w+31.
   __syncwarp();
   const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(done, 0, abort_flag));
+  float* stg = reinterpret_cast<float*>(smem);             // [TM][EP_LD]
   if (ok) {
     tc::fence_after_sync();
-    const int row = m0 + warp * 32 + lane;
-    const bool rv = row < R;
-    float* wrow = Wk + int64_t(rv ? row : 0) * C;
+    float* srow = stg + (warp * 32 + lane) * EP_LD;
     for (int c = 0; c < TN / 16; ++c) {
       uint32_t v[16];
       tc::tmem_ld_32x16(tmem + (uint32_t(warp * 32) << 16) + uint32_t(c * 16), v);
       tc::tmem_ld_wait();
-      const int col = n0 + c * 16;
-      if (!rv) continue;
-      if (vec && col + 16 <= cend) {
-        float4* p = reinterpret_cast<float4*>(wrow + col);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float4 w = p[q];
-          w.x -= __uint_as_float(v[4 * q + 0]);
-          w.y -= __uint_as_float(v[4 * q + 1]);
-          w.z -= __uint_as_float(v[4 * q + 2]);
-          w.w -= __uint_as_float(v[4 * q + 3]);
-          p[q] = w;
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<float4*>(srow + c * 16 + 4 * q) =
+            make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                        __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3]));
+    }
+  }
+  __syncthreads();
+  if (ok) {
+    // warp w: rows 32w .. 32w+31, eight at a time; lane l: column quads l and
+    // l + 32 of each row.  A batch's loads are all issued before its stores (the
+    // compiler cannot reorder a load of one row past the store of another).
+    constexpr int RB = 8;
+    const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < 32; i0 += RB) {
+      float4 w[RB][2];
+#pragma unroll
+      for (int j = 0; j < RB; ++j) {
+        const int row = m0 + warp * 32 + i0 + j;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int col = n0 + 4 * (lane + 32 * h);
+          w[j][h] = (vec && row < R && col + 4 <= cend)
+                        ? *reinterpret_cast<const float4*>(Wk + int64_t(row) * C + col)
+                        : zero4;
         }
-      } else {
+      }
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (col + q < cend) wrow[col + q] -= __uint_as_float(v[q]);
+      for (int j = 0; j < RB; ++j) {
+        const int rr = warp * 32 + i0 + j, row = m0 + rr;
+        if (row >= R) continue;
+        float* wrow = Wk + int64_t(row) * C;
+        const float* srow = stg + rr * EP_LD;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int cq = lane + 32 * h, col = n0 + 4 * cq;
+          const float4 a = *reinterpret_cast<const float4*>(srow + 4 * cq);
+          if (vec && col + 4 <= cend) {
+            float4 x = w[j][h];
+            x.x -= a.x; x.y -= a.y; x.z -= a.z; x.w -= a.w;
+            *reinterpret_cast<float4*>(wrow + col) = x;
+          } else {
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (col + q < cend) wrow[col + q] -= av[q];
+          }
+        }
       }
     }
   }
