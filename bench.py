@@ -209,21 +209,28 @@ def run_ours(args, rank, world, local_rank):
         layers.append(b)
 
     hess_ev = []
+    phase_ev = []   # per layer: events around hessian / prepare / quantize / pack
 
     def step(record=False):
         for b in layers:
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
             if record:
-                e0 = torch.cuda.Event(enable_timing=True)
-                e1 = torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
+                ev[0].record(stream)
             G.gptq_hessian_accumulate(b["H"], 0, b["X"], b["status"], stream)
             if record:
-                e1.record(stream)
-                hess_ev.append((e0, e1, b["X"].shape[0], b["C"]))
+                ev[1].record(stream)
+                hess_ev.append((ev[0], ev[1], b["X"].shape[0], b["C"]))
             G.gptq_prepare(b["H"], cfg, b["U"], b["perm"], b["wsp"], b["status"], stream)
+            if record:
+                ev[2].record(stream)
             G.gptq_quantize_layer(b["W"], b["U"], b["perm"], cfg, b["codes"], b["scales"],
                                   b["zeros"], b["g_idx"], b["losses"], b["wsq"], b["status"], stream)
+            if record:
+                ev[3].record(stream)
             G.gptq_pack(b["codes"], cfg.bits, b["packed"], stream)
+            if record:
+                ev[4].record(stream)
+                phase_ev.append((b["R"], b["C"], ev))
 
     import torch.distributed as dist
 
@@ -256,6 +263,26 @@ def run_ours(args, rank, world, local_rank):
     cl = clocks.stop()
     ms = t0.elapsed_time(t1)
     hess_ms = sum(a.elapsed_time(b) for a, b, _, _ in hess_ev)
+    # per phase, summed over the layers of one step, and each phase's useful
+    # flop rate (Hessian N C (C+1); Cholesky + triangular inverse 2/3 C^3; lazy
+    # trailing update R C^2)
+    names = ("hessian", "prepare", "quantize", "pack")
+    tot = {n: 0.0 for n in names}
+    flop = {"hessian": 0.0, "prepare": 0.0, "quantize": 0.0}
+    for (R_, C_, ev), (_, _, m, _) in zip(phase_ev, hess_ev):
+        for i, n in enumerate(names):
+            tot[n] += ev[i].elapsed_time(ev[i + 1])
+        flop["hessian"] += float(m) * C_ * (C_ + 1)
+        flop["prepare"] += 2.0 * C_ ** 3 / 3.0
+        flop["quantize"] += float(R_) * C_ * C_
+    basis = {"hessian": "N*C*(C+1)", "prepare": "2/3*C^3",
+             "quantize": "R*C^2 (lazy trailing update; the phase also runs the sweep)"}
+    phases = {}
+    for n in names:
+        phases[n] = {"ms_per_step": tot[n] / args.steps}
+        if n in flop and tot[n] > 0:
+            phases[n]["tflops"] = flop[n] / (tot[n] * 1e-3) / 1e12
+            phases[n]["flop"] = basis[n]
     hess_flop = sum(float(m) * C * (C + 1) for _, _, m, C in hess_ev)
     n_hess = len(hess_ev)
 
@@ -313,6 +340,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": f"{wl.xdtype} inputs, f32 accumulate/solve",
         "data": "synthetic (seeded; stands in for the pages' calibration text)",
         "config": workload_config(wl, world),
+        "phases": phases,
         "hessian": {"ms_per_launch": hess_ms / max(n_hess, 1), "tflops": achieved,
                     "launches": n_hess},
         "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",

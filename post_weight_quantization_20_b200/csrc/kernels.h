@@ -24,13 +24,14 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
                          uint8_t* codes, float* scales, float* zeros, int32_t* g_idx,
                          float* losses, void* ws, int32_t* status);
 
-// trailing_tc.cu: W[:, e:cend] -= (Ehi + Elo) * U[i0:i0+128, e:cend] on tcgen05
-// (3xTF32), with U given as its transposed split Ut_hi + Ut_lo (split_tf32_t)
+// trailing_tc.cu: W[:, e:cend] -= (Ehi + Elo)[:, kE0:kE0+K] * U[i0:i0+K, e:cend] on
+// tcgen05 (3xTF32), with U given as its transposed split Ut_hi + Ut_lo
+// (split_tf32_t) and the errors as column windows of rows x ldE buffers
 bool trailing_tc_supported(int C);
 gptq_status split_tf32_t(cudaStream_t st, const float* U, int C, float* hi, float* lo);
-gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e, int cend,
-                               const float* Ehi, const float* Elo, const float* Uthi,
-                               const float* Utlo, int32_t* status);
+gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int K, int e,
+                               int cend, const float* Ehi, const float* Elo, int ldE, int kE0,
+                               const float* Uthi, const float* Utlo, int32_t* status);
 
 // pack.cu
 gptq_status pack_run(cudaStream_t st, const uint8_t* codes, int64_t R, int64_t C, int bits,

@@ -10,6 +10,7 @@
 // The factorization runs on a Cp x Cp copy (Cp = C rounded up to 64) whose
 // padding is the identity, so every 64-block is full.
 #include <algorithm>
+#include <climits>
 
 #include "common.cuh"
 #include "gemm_f32.cuh"
@@ -20,10 +21,13 @@ namespace gptq {
 
 constexpr int NB = 64;  // diagonal block of the factorization
 
+constexpr int MAX_FACTOR_GRID = 1024;   // CTAs of the persistent factorization (at most)
+
 struct PrepLayout {
   int Cp, nblk;
   float *A, *Bx, *T, *diag, *lam;
   int32_t* cnt;
+  int32_t* smid;   // [MAX_FACTOR_GRID]: the SM each CTA of the factorization runs on
 };
 
 static PrepLayout prep_layout(void* ws, int64_t C) {
@@ -38,6 +42,7 @@ static PrepLayout prep_layout(void* ws, int64_t C) {
   L.diag = reinterpret_cast<float*>(p);         p += align256(size_t(C) * 4);
   L.lam = reinterpret_cast<float*>(p);          p += 256;
   L.cnt = reinterpret_cast<int32_t*>(p);        p += align256(size_t(C) * 4);
+  L.smid = reinterpret_cast<int32_t*>(p);       p += align256(size_t(MAX_FACTOR_GRID) * 4);
   return L;
 }
 
@@ -45,7 +50,7 @@ size_t prepare_ws_bytes(int64_t C) {
   const int64_t nblk = (C + NB - 1) / NB, Cp = nblk * NB;
   const size_t cp2 = size_t(Cp) * Cp * sizeof(float);
   return 2 * align256(cp2) + align256(size_t(nblk) * NB * NB * 4) + align256(size_t(C) * 4) +
-         256 + align256(size_t(C) * 4);
+         256 + align256(size_t(C) * 4) + align256(size_t(MAX_FACTOR_GRID) * 4);
 }
 
 // lambda = damp * mean(diag H); flags a non-finite diagonal.
@@ -370,6 +375,7 @@ struct FactorArgs {
   unsigned* bar;       // monotonically increasing arrival counter (zeroed before launch)
   int* abort_flag;     // set when a barrier gave up
   int32_t* status;
+  int32_t* smid;       // [gridDim.x]
 };
 
 constexpr uint32_t BARRIER_SPIN_LIMIT = 1u << 24;
@@ -542,10 +548,32 @@ __device__ __forceinline__ void run_tiles64(int t, int step, int end, const Map&
 __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs a) {
   // one buffer: GEMM chunks, or the tiles of the diagonal factor
   __shared__ __align__(16) float sm[GM_SMEM_FLOATS];
+  __shared__ int idle_cta;
   const int64_t lda = a.lda;
   unsigned epoch = 0;
+  if (threadIdx.x == 0) {
+    unsigned id;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(id));
+    a.smid[blockIdx.x] = int32_t(id);
+  }
   if (blockIdx.x == 0) diag_factor(a.A, lda, 0, a.T, a.status, sm);
   if (!grid_barrier(a, epoch)) return;
+  // CTA 0 carries the serial chain (the next diagonal block's update and factor).
+  // A CTA that shares its SM would take half of its issue slots, so that CTA, if
+  // there is one, sits the tile phases out; every CTA finds it by the same scan.
+  if (threadIdx.x == 0) idle_cta = INT_MAX;
+  __syncthreads();
+  {
+    const volatile int32_t* sid = a.smid;
+    const int32_t s0 = sid[0];
+    for (int b = 1 + int(threadIdx.x); b < int(gridDim.x); b += blockDim.x)
+      if (sid[b] == s0) atomicMin(&idle_cta, b);
+  }
+  __syncthreads();
+  const int idle = idle_cta == INT_MAX ? -1 : idle_cta;
+  const int nw = int(gridDim.x) - (idle >= 0 ? 1 : 0);                 // working CTAs
+  const int rank = int(blockIdx.x) - (idle >= 0 && int(blockIdx.x) > idle ? 1 : 0);
+  const bool works = int(blockIdx.x) != idle;
   for (int k = 0; k < a.nblk; ++k) {
     const int k0 = k * NB;
     const float* Tk = a.T + size_t(k) * NB * NB;
@@ -571,7 +599,7 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
       T.acc = false;
       return T;
     };
-    run_tiles64(blockIdx.x, gridDim.x, nr + k + 1, phase_a, sm);
+    if (works) run_tiles64(rank, nw, nr + k + 1, phase_a, sm);
     if (!grid_barrier(a, epoch)) return;
     if (rest == 0) break;
     // phase B: A[k0+64:, k0+64:] -= P P^T (lower tiles) and
@@ -605,9 +633,9 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
       run_tiles64(0, 1, 1, phase_b, sm);     // the next diagonal block first
       diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, sm);
     }
-    const int workers = gridDim.x > 1 ? gridDim.x - 1 : 1;
-    const int first = gridDim.x > 1 ? int(blockIdx.x) - 1 : 0;
-    if (gridDim.x == 1 || blockIdx.x > 0) run_tiles64(1 + first, workers, n_total, phase_b, sm);
+    const int workers = nw > 1 ? nw - 1 : 1;
+    const int first = nw > 1 ? rank - 1 : 0;
+    if (works && (nw == 1 || blockIdx.x > 0)) run_tiles64(1 + first, workers, n_total, phase_b, sm);
     if (!grid_barrier(a, epoch)) return;
   }
 }
@@ -647,7 +675,7 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
   unsigned* bar = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(L.lam) + 64);
   int* abort_flag = reinterpret_cast<int*>(reinterpret_cast<char*>(L.lam) + 128);
   GPTQ_CUDA(cudaMemsetAsync(reinterpret_cast<char*>(L.lam) + 64, 0, 128, st));
-  FactorArgs fa{L.A, L.Bx, L.T, Cp, L.nblk, bar, abort_flag, status};
+  FactorArgs fa{L.A, L.Bx, L.T, Cp, L.nblk, bar, abort_flag, status, L.smid};
   int per_sm = 0;
   GPTQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_factor_persistent,
                                                           GM_THREADS, 0));
@@ -656,7 +684,7 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
   // enough CTAs for the largest phase, at most what can be co-resident
   const int nr0 = Cp / NB - 1;
   const int most = std::max(1, std::max(nr0 * (nr0 + 1) / 2 + nr0, nr0 + Cp / NB));
-  const int grid = std::min(std::min(per_sm, 2) * sms, most + 1);
+  const int grid = std::min(std::min(std::min(per_sm, 2) * sms, most + 1), MAX_FACTOR_GRID);
   void* args[] = {&fa};
   GPTQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_factor_persistent), dim3(grid),
                                         dim3(GM_THREADS), args, 0, st));

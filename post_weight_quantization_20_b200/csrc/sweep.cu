@@ -3,8 +3,9 @@
 //
 // Data layout in HBM (workspace):
 //   Wk    rows x C fp32   working copy of W in sweep order (columns gathered by perm)
-//   Err   2 x rows x 128 fp32 scaled errors (w - Q)/U[q][q] of a panel, split hi + lo,
-//         double-buffered by panel parity
+//   Err   rows x 2048 fp32 (hi and lo parts) scaled errors (w - Q)/U[q][q]; panel p
+//         writes columns 128 (p % 16) .. +128, so the errors of two consecutive
+//         blocks of eight panels are held at once
 //   cp    rows x C u8     codes in sweep order
 //   lpart tiles x C fp32  per-row-tile partial column losses (summed in finalize)
 //
@@ -24,6 +25,9 @@
 namespace gptq {
 
 constexpr int SW_B = 128;                 // panel width (columns)
+constexpr int SW_B2 = 1024;               // second level of the lazy update (8 panels)
+constexpr int SW_ESLOTS = 2 * SW_B2 / SW_B;
+constexpr int SW_LDERR = SW_ESLOTS * SW_B; // row stride of the error buffers
 constexpr int SW_TPR = 8;                 // threads per row
 constexpr int SW_CPT = SW_B / SW_TPR;     // panel columns owned by one thread (16)
 constexpr int SW_ROWS = 16;               // rows per CTA
@@ -35,8 +39,8 @@ constexpr int SW_SMEM = (SW_B * SW_LDU + SW_B + SW_ROWS * SW_LDE) * 4;
 
 struct QuantLayout {
   float* Wk;
-  float* Ehi[2];
-  float* Elo[2];
+  float* Ehi;    // rows x SW_LDERR
+  float* Elo;
   uint8_t* cp;
   float* lpart;
   float* Uhi;
@@ -49,10 +53,8 @@ static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
   L.tiles = int((R + SW_ROWS - 1) / SW_ROWS);
   char* p = static_cast<char*>(ws);
   L.Wk = reinterpret_cast<float*>(p);    p += align256(size_t(R) * C * 4);
-  for (int b = 0; b < 2; ++b) {
-    L.Ehi[b] = reinterpret_cast<float*>(p); p += align256(size_t(R) * SW_B * 4);
-    L.Elo[b] = reinterpret_cast<float*>(p); p += align256(size_t(R) * SW_B * 4);
-  }
+  L.Ehi = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_LDERR * 4);
+  L.Elo = reinterpret_cast<float*>(p);   p += align256(size_t(R) * SW_LDERR * 4);
   L.cp = reinterpret_cast<uint8_t*>(p);  p += align256(size_t(R) * C);
   L.lpart = reinterpret_cast<float*>(p); p += align256(size_t(L.tiles) * C * 4);
   L.Uhi = reinterpret_cast<float*>(p);   p += align256(size_t(C) * C * 4);
@@ -62,7 +64,7 @@ static QuantLayout quant_layout(void* ws, int64_t R, int64_t C) {
 
 size_t quantize_ws_bytes(int64_t R, int64_t C, const gptq_config&) {
   const int64_t tiles = (R + SW_ROWS - 1) / SW_ROWS;
-  return align256(size_t(R) * C * 4) + 4 * align256(size_t(R) * SW_B * 4) +
+  return align256(size_t(R) * C * 4) + 2 * align256(size_t(R) * SW_LDERR * 4) +
          align256(size_t(R) * C) + align256(size_t(tiles) * C * 4) +
          2 * align256(size_t(C) * C * 4) + 256;
 }
@@ -126,6 +128,7 @@ __global__ void __launch_bounds__(SW_THREADS)
 k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits, int g, int sym,
               float* scales, float* zeros, int G, uint8_t* cp, float* Ehi, float* Elo,
               float* lpart, const float* Eph, const float* Epl, int ip) {
+  constexpr int ldE = SW_LDERR;   // row stride of the error buffers
   extern __shared__ __align__(16) float sm[];
   float* Us = sm;                       // SW_B x SW_LDU
   float* dinv = Us + SW_B * SW_LDU;     // SW_B
@@ -188,8 +191,8 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
         const int e4 = tid + SW_THREADS * x, rr = e4 / (SW_B / 4), k = 4 * (e4 % (SW_B / 4));
         const int row = blockIdx.x * SW_ROWS + rr;
         const float4 zero4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        hq[x] = row < R ? *reinterpret_cast<const float4*>(Eph + int64_t(row) * SW_B + k) : zero4;
-        lq[x] = row < R ? *reinterpret_cast<const float4*>(Epl + int64_t(row) * SW_B + k) : zero4;
+        hq[x] = row < R ? *reinterpret_cast<const float4*>(Eph + int64_t(row) * ldE + k) : zero4;
+        lq[x] = row < R ? *reinterpret_cast<const float4*>(Epl + int64_t(row) * ldE + k) : zero4;
       }
       load_ublock(ip, SW_B);
 #pragma unroll
@@ -298,8 +301,8 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
       hv[jj] = __uint_as_float(__float_as_uint(e[jj]) & 0xFFFFE000u);
       lv[jj] = e[jj] - hv[jj];
     }
-    float4* hrow = reinterpret_cast<float4*>(Ehi + int64_t(r) * SW_B + t * SW_CPT);
-    float4* lrw = reinterpret_cast<float4*>(Elo + int64_t(r) * SW_B + t * SW_CPT);
+    float4* hrow = reinterpret_cast<float4*>(Ehi + int64_t(r) * ldE + t * SW_CPT);
+    float4* lrw = reinterpret_cast<float4*>(Elo + int64_t(r) * ldE + t * SW_CPT);
 #pragma unroll
     for (int q = 0; q < SW_CPT / 4; ++q) {
       hrow[q] = make_float4(hv[4 * q], hv[4 * q + 1], hv[4 * q + 2], hv[4 * q + 3]);
@@ -376,17 +379,25 @@ static cudaStream_t side_stream(gptq_status& err) {
   return streams[dev];
 }
 
-// The panels with the lazy trailing update split in two (a lookahead of one
-// panel).  The sweep of panel p first applies panel p-1's update to its own
-// columns (in fp32, from the errors p-1 left in its buffer), then sweeps; a side
-// stream applies panel p's update to the columns from panel p+2 on.  Order: the
-// side update of p starts after the sweep of p; the sweep of p waits for the side
-// update of p-2, the last one that writes its columns (side updates run in panel
-// order on the side stream).  Panel errors alternate between two buffers, and the
-// sweep of p+2, which overwrites p's, waits for the side update of p, the last
-// reader.  The caller's stream joins the side stream before returning (event
-// fork/join, so the call can be stream-captured).  Every column receives its
-// panel updates in panel order, so results are deterministic.
+// The panels, with the lazy trailing update in two levels and a lookahead of one
+// panel.  Panel p of block S (eight panels, SW_B2 columns, ending at column S_end):
+//   * the sweep of p first applies panel p-1's update to its own columns (in
+//     fp32, from the errors p-1 left in its slot), then sweeps;
+//   * a side stream applies p's update (K = 128) to the columns from panel p+2
+//     up to and including the first panel after block S;
+//   * after the last panel of S, the side stream applies the update of all of S
+//     (K = 1024) to the columns after that.
+// So every panel receives exactly one update from every earlier panel, and the
+// far columns are rewritten once per block instead of once per panel.  Order:
+// side work for p starts after the sweep of p; the sweep of p waits for the side
+// work enqueued after the sweep of p-2, which includes every side update that
+// writes p's columns (side work runs in panel order on one stream).  Panel p's
+// errors live in slot p % 16 of the error buffers; the slot is rewritten by the
+// sweep of p+16, after the side work of p+14, so after every reader (the sweep
+// of p+1 and the side updates of p and of its block).  The caller's stream joins
+// the side stream before returning (event fork/join, so the call can be
+// stream-captured).  Every column receives its updates in panel order, so
+// results are deterministic.
 static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R, int C,
                                    const float* U, const gptq_config& cfg, int g, int G,
                                    float* scales, float* zeros, int32_t* status) {
@@ -407,29 +418,38 @@ static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R,
   // fork: the side stream starts after everything the caller enqueued so far
   ce = cudaEventRecord(swept, st);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
-  bool upd[2] = {false, false};   // updated[b] holds the side update of an earlier panel
-  const int np = (C + SW_B - 1) / SW_B;
+  bool upd[2] = {false, false};   // updated[b] holds the side work of an earlier panel
+  const int np = (C + SW_B - 1) / SW_B, per = SW_B2 / SW_B;
   for (int p = 0; p < np && ce == cudaSuccess && err == GPTQ_OK; ++p) {
     const int i0 = p * SW_B, nb = min(SW_B, C - i0), b = p & 1;
-    if (upd[b]) {   // the side update of p-2
+    if (upd[b]) {   // the side work of p-2
       ce = cudaStreamWaitEvent(st, ev[1 + b], 0);
       if (ce != cudaSuccess) break;
       upd[b] = false;
     }
-    const int pb = (p - 1) & 1;
+    const int slot = p % SW_ESLOTS, pslot = (p + SW_ESLOTS - 1) % SW_ESLOTS;
     k_sweep_panel<<<L.tiles, SW_THREADS, SW_SMEM, st>>>(
-        L.Wk, R, C, i0, nb, U, cfg.bits, g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[b], L.Elo[b],
-        L.lpart, L.Ehi[pb], L.Elo[pb], p > 0 ? i0 - SW_B : -1);
+        L.Wk, R, C, i0, nb, U, cfg.bits, g, cfg.sym, scales, zeros, G, L.cp, L.Ehi + slot * SW_B,
+        L.Elo + slot * SW_B, L.lpart, L.Ehi + pslot * SW_B, L.Elo + pslot * SW_B,
+        p > 0 ? i0 - SW_B : -1);
     note_launch();
     ce = cudaGetLastError();
     if (ce != cudaSuccess) break;
-    const int e = i0 + nb + SW_B;   // the side update covers columns from panel p+2 on
-    if (e >= C) continue;
+    const int S0 = (p / per) * SW_B2, S_end = min(S0 + SW_B2, C);
+    const bool last = (p % per == per - 1) || p == np - 1;
+    const int e1 = i0 + nb + SW_B, c1 = min(S_end + SW_B, C);   // panel level
+    const int e2 = S_end + SW_B;                                 // block level
+    const bool lvl1 = e1 < c1, lvl2 = last && e2 < C;
+    if (!lvl1 && !lvl2) continue;
     ce = cudaEventRecord(swept, st);
     if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
     if (ce != cudaSuccess) break;
-    err = trailing_update_tc(side, L.Wk, R, C, i0, e, C, L.Ehi[b], L.Elo[b], L.Uhi, L.Ulo,
-                             status);
+    if (lvl1)
+      err = trailing_update_tc(side, L.Wk, R, C, i0, SW_B, e1, c1, L.Ehi, L.Elo, SW_LDERR,
+                               slot * SW_B, L.Uhi, L.Ulo, status);
+    if (err == GPTQ_OK && lvl2)
+      err = trailing_update_tc(side, L.Wk, R, C, S0, S_end - S0, e2, C, L.Ehi, L.Elo, SW_LDERR,
+                               ((p / per) % 2) * SW_B2, L.Uhi, L.Ulo, status);
     if (err != GPTQ_OK) break;
     ce = cudaEventRecord(ev[1 + b], side);
     upd[b] = ce == cudaSuccess;
@@ -469,14 +489,13 @@ gptq_status quantize_run(cudaStream_t st, const void* W, int wdt, int R, int C, 
     for (int i0 = 0; i0 < C; i0 += SW_B) {
       const int nb = min(SW_B, C - i0);
       GPTQ_LAUNCH(k_sweep_panel, L.tiles, SW_THREADS, SW_SMEM, st, L.Wk, R, C, i0, nb, U, cfg.bits,
-                  g, cfg.sym, scales, zeros, G, L.cp, L.Ehi[0], L.Elo[0], L.lpart, nullptr,
-                  nullptr, -1);
+                  g, cfg.sym, scales, zeros, G, L.cp, L.Ehi, L.Elo, L.lpart, nullptr, nullptr, -1);
       const int e = i0 + nb;
       if (e < C) {
         // W[:, e:] -= Err[:, 0:nb] * U[i0:e, e:]
-        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Ehi[0], SW_B, 1, U + int64_t(i0) * C + e, C,
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Ehi, SW_LDERR, 1, U + int64_t(i0) * C + e, C,
                           1, 1.f, L.Wk + e, C, 0));
-        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Elo[0], SW_B, 1, U + int64_t(i0) * C + e, C,
+        GPTQ_TRY(gemm_f32(st, R, C - e, nb, -1.f, L.Elo, SW_LDERR, 1, U + int64_t(i0) * C + e, C,
                           1, 1.f, L.Wk + e, C, 0));
       }
     }

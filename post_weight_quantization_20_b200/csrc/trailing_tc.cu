@@ -1,8 +1,8 @@
 // Lazy trailing update on the tensor cores, GPTQ量化算法深度解析 §2.4:
-//   W[:, e:cend] -= Err * U[i0:e, e:cend]
-// Err (rows x 128) holds the scaled errors of the panel just swept; a call may
-// cover any column range after the panel (the sweep updates the next panel's
-// columns first and the rest concurrently).  The product
+//   W[:, e:cend] -= Err * U[i0:i0+K, e:cend]
+// Err (rows x K, a column window of a rows x ldE buffer) holds the scaled errors
+// of the panel just swept (K = 128) or of a block of eight panels (K = 1024, the
+// second level of the lazy update); a call may cover any column range after them.  The product
 // is fp32-faithful by a 3xTF32 split: x = hi + lo with hi = x with its low 13
 // mantissa bits cleared (exact in tf32) and lo = x - hi, and
 //   Err * U ~= Err_hi U_hi + Err_hi U_lo + Err_lo U_hi
@@ -10,7 +10,7 @@
 // U is split and transposed once per layer into Ut_hi / Ut_lo (C x C, Ut[n][k] =
 // U[k][n]) so that both operands are K-major.
 //
-// One CTA per 128 x 256 output tile; K = 128 in four 32-deep stages, two stages
+// One CTA per 128 x 256 output tile; K in 32-deep stages, two stages
 // in flight (96 KB each: Err hi+lo and Ut hi+lo K-major boxes of 32 K-values x
 // 128 rows, 128-byte swizzled by TMA).  Warp 0 issues TMA, warp 1 issues tcgen05.mma
 // kind::tf32 (M=128, N=256, K=8) into one 256-column TMEM accumulator, then all
@@ -24,7 +24,7 @@
 namespace gptq {
 namespace {
 
-constexpr int TM = 128, TN = 256, TK = 32, NSTAGE_K = 4;   // K = 128 per panel
+constexpr int TM = 128, TN = 256, TK = 32;   // K = 32 per stage, K / 32 stages
 constexpr int A_BOX = TM * TK * 4;                         // 16 KB: 128 rows x 128 B
 constexpr int B_BOX = 128 * TK * 4;                        // 16 KB: 128 N-rows x 128 B
 constexpr int STAGE = 2 * A_BOX + 2 * (TN / 128) * B_BOX;  // 96 KB
@@ -37,8 +37,8 @@ static_assert(TM * EP_LD * 4 <= BUFS * STAGE, "the stage buffers hold the accumu
 __global__ void __launch_bounds__(THREADS, 1)
 k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ CUtensorMap elo,
               const __grid_constant__ CUtensorMap uhi, const __grid_constant__ CUtensorMap ulo,
-              float* Wk, int R, int C, int i0, int e, int cend, uint32_t idesc, int vec,
-              int32_t* status) {
+              float* Wk, int R, int C, int i0, int e, int cend, int kE0, int nk,
+              uint32_t idesc, int vec, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -69,14 +69,14 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < NSTAGE_K; ++s) {
+    for (int s = 0; s < nk; ++s) {
       const int b = s % BUFS;
       if (s >= BUFS && !tc::mbar_wait(empty + b, ((s / BUFS) - 1) & 1, abort_flag)) break;
       uint8_t* st = smem + b * STAGE;
       tc::mbar_expect_tx(full + b, STAGE);
       const int k0 = s * TK;
-      tc::tma_load_2d(st, &ehi, k0, m0, full + b);
-      tc::tma_load_2d(st + A_BOX, &elo, k0, m0, full + b);
+      tc::tma_load_2d(st, &ehi, kE0 + k0, m0, full + b);
+      tc::tma_load_2d(st + A_BOX, &elo, kE0 + k0, m0, full + b);
       uint8_t* bh = st + 2 * A_BOX;
       uint8_t* bl = bh + (TN / 128) * B_BOX;
       for (int q = 0; q < TN / 128; ++q) {
@@ -86,7 +86,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
     }
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
-    for (int s = 0; s < NSTAGE_K && ok; ++s) {
+    for (int s = 0; s < nk && ok; ++s) {
       const int b = s % BUFS;
       if (!tc::mbar_wait(full + b, (s / BUFS) & 1, abort_flag)) { ok = false; break; }
       tc::fence_after_sync();
@@ -240,13 +240,15 @@ gptq_status split_tf32_t(cudaStream_t st, const float* U, int C, float* hi, floa
   return GPTQ_OK;
 }
 
-gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int e, int cend,
-                               const float* Ehi, const float* Elo, const float* Uthi,
-                               const float* Utlo, int32_t* status) {
-  if (e >= cend || cend > C || R <= 0) return GPTQ_OK;
+gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0, int K, int e,
+                               int cend, const float* Ehi, const float* Elo, int ldE, int kE0,
+                               const float* Uthi, const float* Utlo, int32_t* status) {
+  if (e >= cend || R <= 0) return GPTQ_OK;
+  if (cend > C || K <= 0 || K % TK || kE0 % TK || kE0 + K > ldE || e < i0 + K)
+    return GPTQ_ERR_INVALID_ARG;
   CUtensorMap mehi, melo, muhi, mulo;
-  if (!encode_2d(&mehi, Ehi, 128, uint64_t(R), 128, TK, TM) ||
-      !encode_2d(&melo, Elo, 128, uint64_t(R), 128, TK, TM) ||
+  if (!encode_2d(&mehi, Ehi, uint64_t(ldE), uint64_t(R), uint64_t(ldE), TK, TM) ||
+      !encode_2d(&melo, Elo, uint64_t(ldE), uint64_t(R), uint64_t(ldE), TK, TM) ||
       !encode_2d(&muhi, Uthi, uint64_t(C), uint64_t(C), uint64_t(C), TK, 128) ||
       !encode_2d(&mulo, Utlo, uint64_t(C), uint64_t(C), uint64_t(C), TK, 128))
     return GPTQ_ERR_UNSUPPORTED;
@@ -257,7 +259,7 @@ gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0,
   GPTQ_CUDA(allow_smem(k_trailing_tc, SMEM));
   dim3 grid((cend - e + TN - 1) / TN, (R + TM - 1) / TM);
   GPTQ_LAUNCH(k_trailing_tc, grid, THREADS, SMEM, st, mehi, melo, muhi, mulo, Wk, R, C, i0, e,
-              cend, idesc, vec, status);
+              cend, kE0, K / TK, idesc, vec, status);
   return GPTQ_OK;
 }
 
