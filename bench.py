@@ -96,21 +96,28 @@ class ClockSampler:
         pr = torch.cuda.get_device_properties(device)
         self.bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
         self.rows = []
+        self.nv = None
         self.thread = None
         self.proc = None
         self.path = None
         self.stop_evt = None
 
-    def _nvml_loop(self, nv, h):
-        bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
-                "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
-                "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
-                "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
-        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-        while not self.stop_evt.is_set():
-            sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+    def _nvml_sample(self):
+        nv, h, mx, bits = self.nv
+        try:
+            sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        except Exception:
+            return
+        try:
             rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-            self.rows.append((float(sm), float(mx), [k for k, b in bits.items() if rs & b]))
+            reasons = [k for k, b in bits.items() if rs & b]
+        except Exception:
+            reasons = ["unreadable"]
+        self.rows.append((sm, mx, reasons))
+
+    def _nvml_loop(self):
+        while not self.stop_evt.is_set():
+            self._nvml_sample()
             self.stop_evt.wait(self.PERIOD_S)
 
     def start(self):
@@ -119,12 +126,21 @@ class ClockSampler:
             import pynvml as nv
             nv.nvmlInit()
             h = nv.nvmlDeviceGetHandleByPciBusId(self.bus.encode())
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self.nv = (nv, h, float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)), bits)
+            self._nvml_sample()                  # one sample at the start of the region
+            if not self.rows:
+                raise RuntimeError("NVML gave no clock reading")
             self.stop_evt = threading.Event()
-            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h), daemon=True)
+            self.thread = threading.Thread(target=self._nvml_loop, daemon=True)
             self.thread.start()
             return
         except Exception:
             self.thread = None
+            self.rows = []
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -139,6 +155,7 @@ class ClockSampler:
         if self.thread is not None:
             self.stop_evt.set()
             self.thread.join(timeout=5)
+            self._nvml_sample()                      # and one at its end
             rows = self.rows
         elif self.proc is not None:
             self.proc.terminate()

@@ -199,6 +199,11 @@ CASES = [
     ("single-row", 1, 300, 2000, S.F16, S.F16, 4, 128, False, True, S.ActSpec(mix_rank=3)),
     ("C203-fallback-paths", 70, 203, 1500, S.F16, S.F16, 4, 0, False, False, S.ActSpec(mix_rank=5)),
     ("tall-1000x640", 1000, 640, 3000, S.BF16, S.BF16, 4, 128, False, True, S.ActSpec(mix_rank=8)),
+    # more than 1024 columns: the second level of the lazy update (one K = 1024
+    # update per block of eight panels) and the panel slots of two blocks
+    ("two-level-1408", 96, 1408, 4000, S.F16, S.F16, 4, 128, False, False, S.ActSpec(mix_rank=6)),
+    ("two-level-ragged-2200-act", 64, 2200, 5000, S.BF16, S.BF16, 4, 64, False, True,
+     S.ActSpec(mix_rank=8)),
 ]
 
 
