@@ -191,6 +191,22 @@ gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits
 gptq_status gptq_prepare_static(const float* H, int64_t cols, const gptq_config* cfg, float* U,
                                 int32_t* perm, int32_t* dev_status, void* stream);
 
+/* Self-test of the failure detection (the pages have no counterpart).  Launches a
+ * kernel whose bounded device wait is made to run out, so that a caller or a test
+ * can check that the wait gives up, OR-s GPTQ_ERR_TIMEOUT into *dev_status and
+ * returns with the context still usable:
+ *   which = GPTQ_SELFTEST_MBARRIER: one CTA waits on a shared-memory mbarrier that
+ *           nothing arrives on (the wait used by the tensor-core pipelines, with a
+ *           shortened limit: well under a second);
+ *   which = GPTQ_SELFTEST_GRID_BARRIER: two CTAs, of which one leaves without
+ *           arriving at the software grid barrier of the persistent factorization;
+ *           the other gives up after that barrier's own limit (about a second).
+ * dev_status must be a device int32.  Returns GPTQ_ERR_INVALID_ARG for another
+ * `which` or a NULL dev_status, GPTQ_ERR_CUDA if the launch fails. */
+#define GPTQ_SELFTEST_MBARRIER 0
+#define GPTQ_SELFTEST_GRID_BARRIER 1
+gptq_status gptq_selftest_timeout(int which, int32_t* dev_status, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* gptq_status_string(int status);
 

@@ -127,6 +127,14 @@ const char* gptq_status_string(int status) {
   }
 }
 
+gptq_status gptq_selftest_timeout(int which, int32_t* dev_status, void* stream) {
+  if (!dev_status) return GPTQ_ERR_INVALID_ARG;
+  if (which == GPTQ_SELFTEST_MBARRIER) return selftest_mbarrier(as_stream(stream), dev_status);
+  if (which == GPTQ_SELFTEST_GRID_BARRIER)
+    return selftest_grid_barrier(as_stream(stream), dev_status);
+  return GPTQ_ERR_INVALID_ARG;
+}
+
 uint64_t gptq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 const char* gptq_last_error(void) { return g_last_error; }

@@ -33,6 +33,10 @@ gptq_status trailing_update_tc(cudaStream_t st, float* Wk, int R, int C, int i0,
                                int cend, const float* Ehi, const float* Elo, int ldE, int kE0,
                                const float* Uthi, const float* Utlo, int32_t* status);
 
+// selftest kernels (prepare.cu holds the grid-barrier one, next to the barrier)
+gptq_status selftest_mbarrier(cudaStream_t st, int32_t* status);
+gptq_status selftest_grid_barrier(cudaStream_t st, int32_t* status);
+
 // pack.cu
 gptq_status pack_run(cudaStream_t st, const uint8_t* codes, int64_t R, int64_t C, int bits,
                      uint32_t* packed);

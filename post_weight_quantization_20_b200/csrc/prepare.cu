@@ -378,7 +378,10 @@ struct FactorArgs {
   int32_t* smid;       // [gridDim.x]
 };
 
-constexpr uint32_t BARRIER_SPIN_LIMIT = 1u << 24;
+// Spins of a grid-barrier wait before it gives up (each a ~64 ns sleep and an
+// acquire load from L2: about a second).  A legitimate wait is at most one phase
+// of tiles, a few milliseconds even at C = 49152.
+constexpr uint32_t BARRIER_SPIN_LIMIT = 1u << 21;
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
   unsigned v;
@@ -408,6 +411,19 @@ __device__ bool grid_barrier(const FactorArgs& a, unsigned& epoch) {
   }
   __syncthreads();
   return ok != 0;
+}
+
+// Self-test: CTA 1 leaves without arriving, so CTA 0's barrier wait runs out (it
+// then sets the abort flag and GPTQ_ERR_TIMEOUT).  The slot holds the counter at
+// +0 and the abort flag at +64; the host zeroes it first.
+__global__ void k_selftest_grid_barrier(unsigned* slot, int32_t* status) {
+  if (blockIdx.x != 0) return;
+  FactorArgs a{};
+  a.bar = slot;
+  a.abort_flag = reinterpret_cast<int*>(reinterpret_cast<char*>(slot) + 64);
+  a.status = status;
+  unsigned epoch = 0;
+  grid_barrier(a, epoch);
 }
 
 // lower-triangular tile t of an nr x nr tile grid: t = tm (tm + 1) / 2 + tn, tn <= tm
@@ -638,6 +654,17 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
     if (works && (nw == 1 || blockIdx.x > 0)) run_tiles64(1 + first, workers, n_total, phase_b, sm);
     if (!grid_barrier(a, epoch)) return;
   }
+}
+
+// the self-test's barrier slot: the library's own, so the call needs no workspace
+__device__ __align__(256) unsigned g_selftest_slot[64];
+
+gptq_status selftest_grid_barrier(cudaStream_t st, int32_t* status) {
+  unsigned* p = nullptr;
+  GPTQ_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_selftest_slot));
+  GPTQ_CUDA(cudaMemsetAsync(p, 0, sizeof(g_selftest_slot), st));
+  GPTQ_LAUNCH(k_selftest_grid_barrier, 2, 32, 0, st, p, status);
+  return GPTQ_OK;
 }
 
 // U[a][b] = Minv[C-1-a][C-1-b] for a <= b, 0 below the diagonal.

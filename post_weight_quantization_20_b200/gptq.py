@@ -36,7 +36,8 @@ _DT = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF
 # every symbol include/gptq.h declares
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare",
            "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count",
-           "gptq_last_error", "gptq_prepare_static")
+           "gptq_last_error", "gptq_prepare_static", "gptq_selftest_timeout")
+GPTQ_SELFTEST_MBARRIER, GPTQ_SELFTEST_GRID_BARRIER = 0, 1
 
 GPTQ_STATIC_MAX_COLS = 1024
 
@@ -90,6 +91,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_launch_count.restype = ctypes.c_uint64
     lib.gptq_prepare_static.argtypes = [vp, i64, cfgp, vp, vp, vp, vp]
     lib.gptq_prepare_static.restype = i32
+    lib.gptq_selftest_timeout.argtypes = [i32, vp, vp]
+    lib.gptq_selftest_timeout.restype = i32
     lib.gptq_last_error.argtypes = []
     lib.gptq_last_error.restype = ctypes.c_char_p
     _lib = lib
@@ -183,6 +186,14 @@ def gptq_pack(codes, bits, packed, stream=None) -> None:
 
 def gptq_status_string(code: int) -> str:
     return load_library().gptq_status_string(int(code)).decode()
+
+
+def gptq_selftest_timeout(which: int, status: torch.Tensor, stream=None) -> None:
+    """Launch the failure-detection self-test `which` (a bounded device wait that is
+    made to run out); it ORs GPTQ_ERR_TIMEOUT into `status` on the device."""
+    _need_cuda(status)
+    _check(load_library().gptq_selftest_timeout(int(which), _ptr(status), _stream(stream)),
+           "gptq_selftest_timeout")
 
 
 def gptq_launch_count() -> int:
