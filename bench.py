@@ -181,6 +181,24 @@ class ClockSampler:
                 "reasons": sorted({x for r in rows for x in r[2]}), "samples": len(rows)}
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(vals, world, device):
+    """Each entry's value on the slowest rank (the job ends when its last rank does)."""
+    if world == 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_ms_per_layer(ms_timed, steps, layers_per_rank, world):
+    """Whole-job ms per layer: every rank quantizes `layers_per_rank` layers per step
+    (replicas, weak scaling), all finished within the slowest rank's time."""
+    return ms_timed / steps / (layers_per_rank * world)
+
+
 # ----------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local_rank):
     import torch
@@ -330,10 +348,7 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(o.nbytes for o in outs)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
-    if world > 1:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
 
     n_layers = len(layers) * world
     peaks = load_peaks()
@@ -345,7 +360,7 @@ def run_ours(args, rank, world, local_rank):
         traffic = HESSIAN_TRAFFIC["bytes_per_token_C3072"] * toks
     out = {
         "metric": METRIC,
-        "value": ms / args.steps / n_layers,
+        "value": job_ms_per_layer(ms, args.steps, len(layers), world),
         "unit": "ms",
         "n_gpus": world,
         "steps": args.steps,
