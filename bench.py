@@ -40,7 +40,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/hessian_tc_C3072_T65536.md (C = 3072, 65536 tokens: 733.8 MB + 139.5 MB),
 # scaled to the bench's 262144-token launch by the token count.  Set to None when
 # the kernel changes until it is captured again.
-HESSIAN_TRAFFIC = {"bytes_per_token_C3072": (733.765120e6 + 139.469824e6) / 65536}
+HESSIAN_TRAFFIC = None
 
 
 def load_peaks():

@@ -11,7 +11,8 @@
 //
 // Precision: the tensor core's fp32 accumulation does not round to nearest, so
 // a long accumulation chain inside TMEM drifts (about 1e-4 relative over 20k
-// tokens).  The MMA therefore accumulates SEG token steps (256 tokens) into one
+// tokens; about 2e-6 with 512-token segments, 1e-6 with 256, at 262144 tokens and
+// C = 3072).  The MMA therefore accumulates SEG token steps (512 tokens) into one
 // of two TMEM buffers, and the epilogue adds each segment into a register
 // accumulator with ordinary round-to-nearest fp32 adds while the MMA fills the
 // other buffer.  At the end of a work item the registers are added into H with
@@ -39,7 +40,7 @@ constexpr int B_BYTES = BN * BK * 2;         // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int BOX_BYTES = 64 * BK * 2;       // one 64-column x 64-token box, 8 KB
 constexpr int THREADS = 320;                 // 2 control warps + 8 epilogue warps
-constexpr int SEG = 4;                       // token steps (of 64) per TMEM segment
+constexpr int SEG = 8;                       // token steps (of 64) per TMEM segment
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 

@@ -276,10 +276,9 @@ k_sweep_panel(float* Wk, int R, int C, int i0, int nb, const float* U, int bits,
       const float x = __shfl_sync(0xffffffffu, w[qq], (lane & ~(SW_TPR - 1)) | c);
       const float cq = fminf(fmaxf(rintf(x * inv_s), cmin), cmax);
       const float err = fmaf(-s, cq, x) * dq;
-      if (t == c) {
-        e[qq] = err;
-        cw[qq >> 2] |= uint32_t(cq + z) << (8 * (qq & 3));
-      }
+      const bool mine = (t == c);
+      e[qq] = mine ? err : e[qq];
+      cw[qq >> 2] |= mine ? (uint32_t(cq + z) << (8 * (qq & 3))) : 0u;
       const float* urow = Us + q * SW_LDU + t * (SW_CPT + 4);
 #pragma unroll
       for (int jj = 0; jj < SW_CPT; jj += 4) {
