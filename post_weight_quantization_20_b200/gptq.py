@@ -241,14 +241,8 @@ def check_status(status: torch.Tensor, where: str = "device") -> None:
         raise GPTQError(code, where)
 
 
-def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | None = None,
-                   chunk_tokens: int | None = None, stream=None, check: bool = True) -> LayerResult:
-    """Quantize one linear layer.  W (rows x cols) and X (tokens x cols, or an
-    iterable of such chunks) are device tensors."""
-    dev = W.device
-    R, C = W.shape
+def _hessian(X, C: int, dev, status, chunk_tokens, stream):
     H = torch.empty(C, C, dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
     n = 0
     chunks = [X] if isinstance(X, torch.Tensor) else X
     for Xc in chunks:
@@ -257,12 +251,21 @@ def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | No
                 n = gptq_hessian_accumulate(H, n, Xc[t0:t0 + chunk_tokens], status, stream)
         else:
             n = gptq_hessian_accumulate(H, n, Xc, status, stream)
+    return H, n
+
+
+def _factor(H, cfg, perm, rows, dev, status, stream):
+    C = H.shape[0]
     U = torch.empty(C, C, dtype=torch.float32, device=dev)
     if perm is None:
         perm = torch.empty(C, dtype=torch.int32, device=dev)
-    ws = alloc_workspace(GPTQ_OP_PREPARE, R, C, cfg, dev)
+    ws = alloc_workspace(GPTQ_OP_PREPARE, rows, C, cfg, dev)
     gptq_prepare(H, cfg, U, perm, ws, status, stream)
-    del ws
+    return U, perm
+
+
+def _sweep(W, U, perm, cfg, dev, status, stream):
+    R, C = W.shape
     G = n_groups(C, cfg.group_size)
     codes = torch.empty(R, C, dtype=torch.uint8, device=dev)
     scales = torch.empty(R, G, dtype=torch.float32, device=dev)
@@ -273,9 +276,64 @@ def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | No
     gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws, status, stream)
     packed = torch.empty(R, packed_words(C, cfg.bits), dtype=torch.int32, device=dev)
     gptq_pack(codes, cfg.bits, packed, stream)
+    return codes, scales, zeros, g_idx, losses, packed
+
+
+def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | None = None,
+                   chunk_tokens: int | None = None, stream=None, check: bool = True) -> LayerResult:
+    """Quantize one linear layer.  W (rows x cols) and X (tokens x cols, or an
+    iterable of such chunks) are device tensors."""
+    dev = W.device
+    R, C = W.shape
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
+    U, perm = _factor(H, cfg, perm, R, dev, status, stream)
+    codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
     if check:
         check_status(status, "quantize_layer")
     return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n)
+
+
+def quantize_layers_shared(Ws, X, cfg: gptq_config, perm: torch.Tensor | None = None,
+                           chunk_tokens: int | None = None, stream=None,
+                           check: bool = True) -> list:
+    """Quantize several linear layers that read the same input (the q/k/v or
+    gate/up projections of one block): one Hessian and one factorization, then one
+    sweep per weight.  Each W is rows_i x cols; the results are those of separate
+    quantize_layer calls on the same X."""
+    Ws = list(Ws)
+    if not Ws:
+        return []
+    dev = Ws[0].device
+    C = Ws[0].shape[1]
+    if any(W.shape[1] != C or W.device != dev for W in Ws):
+        raise ValueError("the weights of a shared-input group need the same cols and device")
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
+    U, perm = _factor(H, cfg, perm, max(W.shape[0] for W in Ws), dev, status, stream)
+    out = []
+    for W in Ws:
+        codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
+        out.append(LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n))
+    if check:
+        check_status(status, "quantize_layers_shared")
+    return out
+
+
+def quantize_rtn(W: torch.Tensor, cfg: gptq_config, stream=None, check: bool = True) -> LayerResult:
+    """Round-to-nearest on the same grids, without error feedback: the sweep with
+    U = I (every off-diagonal of U is zero, so no error is fed forward; the
+    per-column losses are then (w - Q)^2 / 2 summed over rows).  Natural column
+    order; act_order in cfg is ignored."""
+    dev = W.device
+    R, C = W.shape
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    U = torch.eye(C, dtype=torch.float32, device=dev)
+    perm = torch.arange(C, dtype=torch.int32, device=dev)
+    codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
+    if check:
+        check_status(status, "quantize_rtn")
+    return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, None, U, 0)
 
 
 # --------------------------------------------------------------------------- host buffers
