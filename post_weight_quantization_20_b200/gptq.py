@@ -10,6 +10,7 @@ library is missing or no CUDA device is present, the calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from dataclasses import dataclass
@@ -241,6 +242,12 @@ def check_status(status: torch.Tensor, where: str = "device") -> None:
         raise GPTQError(code, where)
 
 
+def _on(stream):
+    """Allocate on the stream the work runs on, so that the caching allocator reuses
+    a buffer (a workspace released before its kernel has run) only in stream order."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _hessian(X, C: int, dev, status, chunk_tokens, stream):
     H = torch.empty(C, C, dtype=torch.float32, device=dev)
     n = 0
@@ -285,10 +292,11 @@ def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | No
     iterable of such chunks) are device tensors."""
     dev = W.device
     R, C = W.shape
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
-    U, perm = _factor(H, cfg, perm, R, dev, status, stream)
-    codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
+    with _on(stream):
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
+        U, perm = _factor(H, cfg, perm, R, dev, status, stream)
+        codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
     if check:
         check_status(status, "quantize_layer")
     return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n)
@@ -308,13 +316,15 @@ def quantize_layers_shared(Ws, X, cfg: gptq_config, perm: torch.Tensor | None = 
     C = Ws[0].shape[1]
     if any(W.shape[1] != C or W.device != dev for W in Ws):
         raise ValueError("the weights of a shared-input group need the same cols and device")
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
-    U, perm = _factor(H, cfg, perm, max(W.shape[0] for W in Ws), dev, status, stream)
     out = []
-    for W in Ws:
-        codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
-        out.append(LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n))
+    with _on(stream):
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
+        U, perm = _factor(H, cfg, perm, max(W.shape[0] for W in Ws), dev, status, stream)
+        for W in Ws:
+            codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status,
+                                                                 stream)
+            out.append(LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n))
     if check:
         check_status(status, "quantize_layers_shared")
     return out
@@ -327,10 +337,11 @@ def quantize_rtn(W: torch.Tensor, cfg: gptq_config, stream=None, check: bool = T
     order; act_order in cfg is ignored."""
     dev = W.device
     R, C = W.shape
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    U = torch.eye(C, dtype=torch.float32, device=dev)
-    perm = torch.arange(C, dtype=torch.int32, device=dev)
-    codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
+    with _on(stream):
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        U = torch.eye(C, dtype=torch.float32, device=dev)
+        perm = torch.arange(C, dtype=torch.int32, device=dev)
+        codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
     if check:
         check_status(status, "quantize_rtn")
     return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, None, U, 0)
