@@ -15,7 +15,10 @@
 // the row applies the rank-1 compensation to its own columns using the panel's
 // U block held in shared memory.  Group grids are warp-shuffle min/max
 // reductions over the row's g columns.  The lazy trailing update
-// W[:, end:] -= Err * U[panel, end:] is a separate GEMM.
+// W[:, end:] -= Err * U[panel, end:] is split three ways (see sweep_lookahead):
+// the next panel's columns inside the next sweep (fp32, before it quantizes),
+// the columns up to the end of the panel's block of eight on the tensor cores,
+// and the columns beyond that once per block (K = 1024).
 #include <algorithm>
 
 #include "common.cuh"
