@@ -151,8 +151,8 @@ gptq_status gptq_prepare(const float* H, int64_t cols, const gptq_config* cfg, f
  *  Streams: part of the lazy update runs on a library-owned side stream (one per
  *  host thread and device) that forks from `stream` at the start of the call and
  *  joins it before the call returns, through events; work enqueued on `stream`
- *  afterwards sees the complete result, and the call can be captured into a CUDA
- *  graph from `stream`.  The per-block update order is fixed, so the outputs are
+ *  afterwards sees the complete result.  (Graph capture of this call has not been
+ *  tested.)  The per-block update order is fixed, so the outputs are
  *  deterministic for a given U and W.
  */
 gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t cols,

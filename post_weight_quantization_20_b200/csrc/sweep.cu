@@ -397,9 +397,8 @@ static cudaStream_t side_stream(gptq_status& err) {
 // errors live in slot p % 16 of the error buffers; the slot is rewritten by the
 // sweep of p+16, after the side work of p+14, so after every reader (the sweep
 // of p+1 and the side updates of p and of its block).  The caller's stream joins
-// the side stream before returning (event fork/join, so the call can be
-// stream-captured).  Every column receives its updates in panel order, so
-// results are deterministic.
+// the side stream before returning (event fork/join).  Every column receives its
+// updates in panel order, so results are deterministic.
 static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R, int C,
                                    const float* U, const gptq_config& cfg, int g, int G,
                                    float* scales, float* zeros, int32_t* status) {
