@@ -119,3 +119,20 @@ def test_binding_refuses_host_tensors():
     X = torch.zeros(8, 4)
     with pytest.raises(ValueError):
         G.gptq_hessian_accumulate(H, 0, X)
+
+
+def test_selftest_rejects_bad_arguments_before_launching():
+    lib = G.load_library()
+    # a NULL status word, or an unknown self-test, is refused on the host
+    assert lib.gptq_selftest_timeout(G.GPTQ_SELFTEST_MBARRIER, None, None) == G.GPTQ_ERR_INVALID_ARG
+    assert lib.gptq_selftest_timeout(7, ctypes.c_void_p(4096), None) == G.GPTQ_ERR_INVALID_ARG
+    assert lib.gptq_selftest_timeout(-1, ctypes.c_void_p(4096), None) == G.GPTQ_ERR_INVALID_ARG
+
+
+def test_binding_helpers_refuse_host_tensors_and_mixed_groups():
+    cfg = G.make_config(4, 128)
+    with pytest.raises(ValueError):
+        G.gptq_selftest_timeout(G.GPTQ_SELFTEST_MBARRIER, torch.zeros(1, dtype=torch.int32))
+    assert G.quantize_layers_shared([], torch.zeros(4, 4), cfg) == []
+    with pytest.raises(ValueError):
+        G.quantize_layers_shared([torch.zeros(2, 4), torch.zeros(2, 5)], torch.zeros(8, 4), cfg)
