@@ -368,3 +368,57 @@ def test_pack_matches_numpy_packbits(bits, cols):
     expect = np.packbits(padded, axis=1, bitorder="little").view("<u4")
     np.testing.assert_array_equal(o.pack(codes, bits), expect)
     np.testing.assert_array_equal(o.unpack(o.pack(codes, bits), bits, cols), codes)
+
+
+# --------------------------------------------------------------------------- degenerate inputs
+def test_dead_input_channel_is_rounded_to_nearest_and_feeds_nothing():
+    """X[:, j] = 0 makes column j of H zero; after damping, Hp couples nothing to j, so
+    U has no off-diagonal entry in row or column j: column j is round-to-nearest of the
+    original weights on the row's grid, and the other columns do not see it."""
+    rng = np.random.default_rng(31)
+    R, C, j = 12, 40, 17
+    X = rng.standard_normal((500, C)) + 0.5 * rng.standard_normal((500, 1))
+    X[:, j] = 0.0
+    H, _ = o.hessian(X)
+    W = 0.02 * rng.standard_normal((R, C))
+    W[:, j] *= 0.1              # never a row's extreme, so the row grids ignore its sign
+    out = o.gptq_quantize(W, H, bits=4, group_size=0, block_size=16)
+    U = out["U"]
+    assert np.all(U[j, j + 1:] == 0.0) and np.all(U[:j, j] == 0.0)
+    s, z, _ = o.grid(W, 4, False)
+    codes_j, Q_j, _ = o.quantize(W[:, j:j + 1], s[:, None], z[:, None], 4)
+    np.testing.assert_array_equal(out["codes"][:, j], codes_j[:, 0])
+    # the other columns do not see column j: flipping its sign (same row grids)
+    # leaves every other code unchanged
+    W2 = W.copy()
+    W2[:, j] = -W[:, j]
+    s2, z2, _ = o.grid(W2, 4, False)
+    assert np.array_equal(s2, s) and np.array_equal(z2, z)
+    out2 = o.gptq_quantize(W2, H, bits=4, group_size=0, block_size=16)
+    others = np.arange(C) != j
+    np.testing.assert_array_equal(out2["codes"][:, others], out["codes"][:, others])
+
+
+def test_all_zero_weight_row_quantizes_to_zero():
+    """A row of zeros has the degenerate range [0, 0], widened to [-1, 1]: every code is
+    the zero-point, Q = 0, and the row adds nothing to the losses."""
+    rng = np.random.default_rng(32)
+    R, C = 6, 32
+    X = rng.standard_normal((300, C))
+    H, _ = o.hessian(X)
+    W = 0.02 * rng.standard_normal((R, C))
+    W[2] = 0.0
+    for bits, sym in ((4, False), (3, True)):
+        out = o.gptq_quantize(W, H, bits=bits, group_size=0, sym=sym, block_size=8)
+        zr = np.ravel(out["zeros"][2])[0]
+        assert np.all(out["codes"][2] == int(zr))
+        assert np.all(out["Q"][2] == 0.0)
+        Wz = np.delete(W, 2, axis=0)
+        ref = o.gptq_quantize(Wz, H, bits=bits, group_size=0, sym=sym, block_size=8)
+        np.testing.assert_allclose(out["losses"], ref["losses"], rtol=1e-12, atol=0)
+
+
+def test_all_zero_hessian_is_not_positive_definite():
+    """H = 0 gives lambda = damp * mean(diag H) = 0 and a zero pivot."""
+    with pytest.raises(o.NotPositiveDefinite):
+        o.gptq_quantize(np.ones((2, 8)), np.zeros((8, 8)), bits=4, group_size=0)
