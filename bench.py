@@ -369,7 +369,7 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": False,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": f"{wl.xdtype} inputs, f32 accumulate/solve",
+        "dtype": "f32",
         "data": "synthetic (seeded; stands in for the pages' calibration text)",
         "config": workload_config(wl, world),
         "phases": phases,
