@@ -125,9 +125,36 @@ def _check(code: int, where: str):
 
 
 def _need_cuda(*ts):
-    for t in ts:
-        if t is not None and not t.is_cuda:
-            raise ValueError("libgptq takes device tensors")
+    devs = {t.device for t in ts if t is not None}
+    if any(d.type != "cuda" for d in devs):
+        raise ValueError("libgptq takes device tensors")
+    if len(devs) > 1:
+        raise ValueError(f"libgptq takes tensors on one device, got {sorted(map(str, devs))}")
+
+
+def _expect(t, name, shape, dtypes, contiguous=True):
+    """The library writes or reads exactly `shape` elements of `t`; check that `t`
+    holds them (it cannot check buffer sizes itself)."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.numel() == 0 and 0 in tuple(shape):
+        return                      # nothing is read or written through it
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _expect_status(status):
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status must be an int32 tensor with at least one element")
+
+
+def _expect_ws(ws):
+    if ws.dtype != torch.uint8 or not ws.is_contiguous():
+        raise ValueError("ws must be a contiguous uint8 tensor")
 
 
 # --------------------------------------------------------------------------- the C calls
@@ -138,10 +165,15 @@ def gptq_workspace_size(op: int, rows: int, cols: int, cfg: gptq_config) -> int:
 def gptq_hessian_accumulate(H: torch.Tensor, n_seen: int, X: torch.Tensor, status=None,
                             stream=None) -> int:
     """H (C x C fp32), X (m x C, row stride X.stride(0)); returns the new token count."""
-    _need_cuda(H, X, status)
-    n = ctypes.c_int64(int(n_seen))
     if X.dim() != 2 or X.stride(1) != 1:
         raise ValueError("X must be 2-D with unit column stride")
+    if X.dtype not in _DT:
+        raise ValueError(f"X must be float32, float16 or bfloat16, got {X.dtype}")
+    C = X.shape[1]
+    _expect(H, "H", (C, C), (torch.float32,))
+    _expect_status(status)
+    _need_cuda(H, X, status)
+    n = ctypes.c_int64(int(n_seen))
     code = load_library().gptq_hessian_accumulate(
         _ptr(H), ctypes.byref(n), _ptr(X), _DT[X.dtype], X.shape[0], X.shape[1], X.stride(0),
         _ptr(status), _stream(stream))
@@ -150,6 +182,12 @@ def gptq_hessian_accumulate(H: torch.Tensor, n_seen: int, X: torch.Tensor, statu
 
 
 def gptq_prepare(H, cfg, U, perm, ws, status=None, stream=None) -> None:
+    C = H.shape[0]
+    _expect(H, "H", (C, C), (torch.float32,))
+    _expect(U, "U", (C, C), (torch.float32,))
+    _expect(perm, "perm", (C,), (torch.int32,))
+    _expect_ws(ws)
+    _expect_status(status)
     _need_cuda(H, U, perm, ws, status)
     code = load_library().gptq_prepare(_ptr(H), H.shape[0], ctypes.byref(cfg), _ptr(U),
                                        _ptr(perm), _ptr(ws), ws.numel() * ws.element_size(),
@@ -160,6 +198,11 @@ def gptq_prepare(H, cfg, U, perm, ws, status=None, stream=None) -> None:
 def gptq_prepare_static(H, cfg, U, perm, status=None, stream=None) -> None:
     """gptq_prepare with the library's built-in scratch array instead of a workspace
     (for callers that cannot allocate; cols <= GPTQ_STATIC_MAX_COLS)."""
+    C = H.shape[0]
+    _expect(H, "H", (C, C), (torch.float32,))
+    _expect(U, "U", (C, C), (torch.float32,))
+    _expect(perm, "perm", (C,), (torch.int32,))
+    _expect_status(status)
     _need_cuda(H, U, perm, status)
     code = load_library().gptq_prepare_static(_ptr(H), H.shape[0], ctypes.byref(cfg), _ptr(U),
                                               _ptr(perm), _ptr(status), _stream(stream))
@@ -168,9 +211,22 @@ def gptq_prepare_static(H, cfg, U, perm, status=None, stream=None) -> None:
 
 def gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws, status=None,
                         stream=None) -> None:
-    _need_cuda(W, U, perm, codes, scales, zeros, g_idx, losses, ws, status)
     if W.dim() != 2 or W.stride(1) != 1:
         raise ValueError("W must be 2-D with unit column stride")
+    if W.dtype not in _DT:
+        raise ValueError(f"W must be float32, float16 or bfloat16, got {W.dtype}")
+    R, C = W.shape
+    G = n_groups(C, cfg.group_size)
+    _expect(U, "U", (C, C), (torch.float32,))
+    _expect(perm, "perm", (C,), (torch.int32,))
+    _expect(codes, "codes", (R, C), (torch.uint8,))
+    _expect(scales, "scales", (R, G), (torch.float32,))
+    _expect(zeros, "zeros", (R, G), (torch.float32,))
+    _expect(g_idx, "g_idx", (C,), (torch.int32,))
+    _expect(losses, "losses", (C,), (torch.float32,))
+    _expect_ws(ws)
+    _expect_status(status)
+    _need_cuda(W, U, perm, codes, scales, zeros, g_idx, losses, ws, status)
     code = load_library().gptq_quantize_layer(
         _ptr(W), _DT[W.dtype], W.shape[0], W.shape[1], W.stride(0), _ptr(U), _ptr(perm),
         ctypes.byref(cfg), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(losses),
@@ -179,6 +235,11 @@ def gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, ws
 
 
 def gptq_pack(codes, bits, packed, stream=None) -> None:
+    if codes.dim() != 2:
+        raise ValueError("codes must be 2-D")
+    R, C = codes.shape
+    _expect(codes, "codes", (R, C), (torch.uint8,))
+    _expect(packed, "packed", (R, packed_words(C, int(bits))), (torch.int32, torch.uint32))
     _need_cuda(codes, packed)
     code = load_library().gptq_pack(_ptr(codes), codes.shape[0], codes.shape[1], int(bits),
                                     _ptr(packed), _stream(stream))
@@ -192,6 +253,7 @@ def gptq_status_string(code: int) -> str:
 def gptq_selftest_timeout(which: int, status: torch.Tensor, stream=None) -> None:
     """Launch the failure-detection self-test `which` (a bounded device wait that is
     made to run out); it ORs GPTQ_ERR_TIMEOUT into `status` on the device."""
+    _expect_status(status)
     _need_cuda(status)
     _check(load_library().gptq_selftest_timeout(int(which), _ptr(status), _stream(stream)),
            "gptq_selftest_timeout")
@@ -397,20 +459,24 @@ def quantize_layer_host(W_host: torch.Tensor, X_host: torch.Tensor, cfg: gptq_co
     dev = torch.device(device) if device is not None else torch.device("cuda")
     comp = stream if stream is not None else torch.cuda.current_stream(dev)
     side = _side_stream(dev)
-    side.wait_stream(comp)          # earlier work on the staging memory is finished
     R, C = W_host.shape
     T = X_host.shape[0]
-    W = torch.empty((R, C), dtype=W_host.dtype, device=dev)
-    stage = [torch.empty((min(chunk_tokens, max(T, 1)), C), dtype=X_host.dtype, device=dev)
-             for _ in range(2)]
+    # Every device buffer is allocated on the compute stream: the caching allocator
+    # hands a freed block out again in that stream's order, and the side stream's
+    # writes into W and the staging buffers are joined into it by events.
+    with torch.cuda.stream(comp):
+        W = torch.empty((R, C), dtype=W_host.dtype, device=dev)
+        stage = [torch.empty((min(chunk_tokens, max(T, 1)), C), dtype=X_host.dtype, device=dev)
+                 for _ in range(2)]
+        H = torch.empty(C, C, dtype=torch.float32, device=dev)
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    side.wait_stream(comp)          # the allocations above are ordered before the copies
     ready = [torch.cuda.Event(), torch.cuda.Event()]
     done = [torch.cuda.Event(), torch.cuda.Event()]
     with torch.cuda.stream(side):
         W.copy_(W_host, non_blocking=True)
     w_ready = torch.cuda.Event()
     w_ready.record(side)
-    H = torch.empty(C, C, dtype=torch.float32, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
     n = 0
     for k, t0 in enumerate(range(0, T, chunk_tokens)):
         m = min(chunk_tokens, T - t0)
@@ -424,9 +490,9 @@ def quantize_layer_host(W_host: torch.Tensor, X_host: torch.Tensor, cfg: gptq_co
         n = gptq_hessian_accumulate(H, n, stage[b][:m], status, comp)
         done[b].record(comp)
     comp.wait_event(w_ready)
-    U = torch.empty(C, C, dtype=torch.float32, device=dev)
-    perm = torch.empty(C, dtype=torch.int32, device=dev)
     with torch.cuda.stream(comp):
+        U = torch.empty(C, C, dtype=torch.float32, device=dev)
+        perm = torch.empty(C, dtype=torch.int32, device=dev)
         wsp = alloc_workspace(GPTQ_OP_PREPARE, R, C, cfg, dev)
         gptq_prepare(H, cfg, U, perm, wsp, status, comp)
         Gn = n_groups(C, cfg.group_size)

@@ -136,3 +136,50 @@ def test_binding_helpers_refuse_host_tensors_and_mixed_groups():
     assert G.quantize_layers_shared([], torch.zeros(4, 4), cfg) == []
     with pytest.raises(ValueError):
         G.quantize_layers_shared([torch.zeros(2, 4), torch.zeros(2, 5)], torch.zeros(8, 4), cfg)
+
+
+def test_binding_checks_buffer_shapes_before_calling_the_library():
+    # the C ABI cannot see buffer sizes, so the binding refuses a buffer that does not
+    # hold what the call reads or writes (checked before the device check, on CPU)
+    cfg = G.make_config(4, 64)
+    R, C = 8, 128
+    W = torch.zeros(R, C, dtype=torch.float16)
+    U = torch.zeros(C, C)
+    perm = torch.zeros(C, dtype=torch.int32)
+    ok = dict(codes=torch.zeros(R, C, dtype=torch.uint8), scales=torch.zeros(R, 2),
+              zeros=torch.zeros(R, 2), g_idx=torch.zeros(C, dtype=torch.int32),
+              losses=torch.zeros(C), ws=torch.zeros(16, dtype=torch.uint8))
+
+    def quantize(**over):
+        a = dict(ok, **over)
+        G.gptq_quantize_layer(W, U, perm, cfg, a["codes"], a["scales"], a["zeros"], a["g_idx"],
+                              a["losses"], a["ws"])
+
+    for name, bad in (("codes", torch.zeros(R, C - 1, dtype=torch.uint8)),
+                      ("codes", torch.zeros(R, C, dtype=torch.int32)),
+                      ("scales", torch.zeros(R, 1)),          # g = 64 gives 2 groups
+                      ("zeros", torch.zeros(R, 2, dtype=torch.float64)),
+                      ("g_idx", torch.zeros(C - 1, dtype=torch.int32)),
+                      ("losses", torch.zeros(C + 1)),
+                      ("codes", torch.zeros(C, R, dtype=torch.uint8).t()),   # not contiguous
+                      ("ws", torch.zeros(4, dtype=torch.float32))):
+        with pytest.raises(ValueError, match=name):
+            quantize(**{name: bad})
+    with pytest.raises(ValueError, match="device tensors"):
+        quantize()                          # shapes fine: refused as host tensors
+    with pytest.raises(ValueError, match="U"):
+        G.gptq_quantize_layer(W, torch.zeros(C, C - 1), perm, cfg, *ok.values())
+    with pytest.raises(ValueError, match="perm"):
+        G.gptq_prepare(U, cfg, torch.zeros(C, C), torch.zeros(C, dtype=torch.int64), ok["ws"])
+    with pytest.raises(ValueError, match="H"):
+        G.gptq_hessian_accumulate(torch.zeros(C, C + 1), 0, torch.zeros(4, C))
+    with pytest.raises(ValueError, match="packed"):
+        G.gptq_pack(ok["codes"], 3, torch.zeros(R, C * 3 // 32 - 1, dtype=torch.int32))
+    with pytest.raises(ValueError, match="status"):
+        G.gptq_selftest_timeout(G.GPTQ_SELFTEST_MBARRIER, torch.zeros(1, dtype=torch.int64))
+    # rows = 0: nothing is written through codes, scales or zeros, so empty ones pass
+    # the shape check (and fail only the device check here)
+    with pytest.raises(ValueError, match="device tensors"):
+        G.gptq_quantize_layer(torch.zeros(0, C, dtype=torch.float16), U, perm, cfg,
+                              torch.zeros(0, dtype=torch.uint8), torch.zeros(0), torch.zeros(0),
+                              ok["g_idx"], ok["losses"], ok["ws"])
