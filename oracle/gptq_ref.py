@@ -367,6 +367,31 @@ def unpack(packed: np.ndarray, bits: int, cols: int) -> np.ndarray:
 
 
 # -----------------------------------------------------------------------------
+# inference side: the layer's product from the stored form
+# [Deep-dive §3.3] (desc_act needs a gather at inference), [gptq-for-llama]
+# "工程细节" (matrix products straight from the packed 4-bit codes)
+# -----------------------------------------------------------------------------
+def dequantize(packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray, g_idx: np.ndarray,
+               bits: int, cols: int) -> np.ndarray:
+    """Q[r, c] = s[r, g] (code[r, c] - z[r, g]) with g = g_idx[c], from the packed codes
+    and the float32 scales / zeros (rows x groups); float64 out, rows x cols."""
+    codes = unpack(packed, bits, cols).astype(np.float64)
+    g = np.asarray(g_idx, dtype=np.int64)
+    s = np.asarray(scales, dtype=np.float32).astype(np.float64)[:, g]
+    z = np.asarray(zeros, dtype=np.float32).astype(np.float64)[:, g]
+    return s * (codes - z)
+
+
+def dequant_matmul(X: np.ndarray, packed: np.ndarray, scales: np.ndarray, zeros: np.ndarray,
+                   g_idx: np.ndarray, bits: int) -> np.ndarray:
+    """Y = X Q^T for activations X (tokens x cols, widened exactly to float64) and the
+    stored layer; Y is tokens x rows, float64."""
+    X = np.asarray(X, dtype=np.float64)
+    Q = dequantize(packed, scales, zeros, g_idx, bits, X.shape[1])
+    return X @ Q.T
+
+
+# -----------------------------------------------------------------------------
 # quality measures  [Deep-dive §2.1]
 # -----------------------------------------------------------------------------
 def half_trace_loss(Wp: np.ndarray, Qp: np.ndarray, Hp: np.ndarray) -> float:

@@ -422,3 +422,54 @@ def test_all_zero_hessian_is_not_positive_definite():
     """H = 0 gives lambda = damp * mean(diag H) = 0 and a zero pivot."""
     with pytest.raises(o.NotPositiveDefinite):
         o.gptq_quantize(np.ones((2, 8)), np.zeros((8, 8)), bits=4, group_size=0)
+
+
+# --------------------------------------------------------------------------- stored form
+def test_dequant_matmul_hand_fixture():
+    """One row of 4-bit codes 0..7 (packed word 0x76543210), scale 0.5, zero 3:
+    Q = 0.5 (c - 3) = -1.5, -1, ..., 2; all-ones input gives 0.5 (28 - 24) = 2, and
+    the input (1, -1, 0, ...) gives -1.5 - (-1) = -0.5."""
+    packed = np.array([[0x76543210]], dtype=np.uint32)
+    g_idx = np.zeros(8, dtype=np.int64)
+    s, z = np.array([[0.5]], np.float32), np.array([[3.0]], np.float32)
+    np.testing.assert_array_equal(o.dequantize(packed, s, z, g_idx, 4, 8)[0],
+                                  [-1.5, -1.0, -0.5, 0.0, 0.5, 1.0, 1.5, 2.0])
+    X = np.array([[1.0] * 8, [1.0, -1.0] + [0.0] * 6])
+    np.testing.assert_array_equal(o.dequant_matmul(X, packed, s, z, g_idx, 4), [[2.0], [-0.5]])
+
+
+@pytest.mark.parametrize("bits,group,sym,act", [(4, 8, False, True), (3, 0, False, False),
+                                                (2, 4, True, True), (3, 16, False, True)])
+def test_stored_form_reproduces_the_sweeps_weights(bits, group, sym, act):
+    """Unpacking the stored codes and gathering each column's grid through g_idx gives
+    exactly the Q the sweep formed column by column in sweep order (a transposed or
+    un-gathered g_idx, or a wrong field offset, breaks the equality under act-order)."""
+    W, X, H, n, *_ = _prep(41 + bits, 7, 32, act=act)
+    out = o.gptq_quantize(W, H, bits, group, sym, act, 0.01, 8)
+    if act:
+        assert not np.all(np.diff(out["g_idx"]) >= 0)       # the gather is not the identity
+    Q = o.dequantize(o.pack(out["codes"], bits), out["scales"], out["zeros"], out["g_idx"],
+                     bits, 32)
+    np.testing.assert_array_equal(Q, out["Q"])
+
+
+def test_dequant_matmul_output_error_is_the_reconstruction_error():
+    """||X W^T - Y||^2 with Y from the stored form equals (n/2) tr((W - Q) H (W - Q)^T)
+    for the undamped H = 2 X^T X / n: the product's orientation pinned through the
+    Hessian route ([Deep-dive §2.1])."""
+    W, X, H, n, *_ = _prep(47, 9, 24, act=True)
+    out = o.gptq_quantize(W, H, 4, 8, False, True, 0.01, 8)
+    Y = o.dequant_matmul(X, o.pack(out["codes"], 4), out["scales"], out["zeros"], out["g_idx"], 4)
+    assert Y.shape == (X.shape[0], W.shape[0])
+    err = float(np.sum((X @ W.T - Y) ** 2))
+    ref = o.reconstruction_error(W, out["Q"], H, n)
+    assert abs(err - ref) <= 1e-9 * ref
+
+
+def test_dequant_matmul_one_hot_inputs_pick_weight_columns():
+    """Token e_c reads column c of Q for every output row."""
+    W, X, H, n, *_ = _prep(53, 5, 16)
+    out = o.gptq_quantize(W, H, 3, 4, False, False, 0.01, 4)
+    Y = o.dequant_matmul(np.eye(16), o.pack(out["codes"], 3), out["scales"], out["zeros"],
+                         out["g_idx"], 3)
+    np.testing.assert_array_equal(Y, out["Q"].T)
