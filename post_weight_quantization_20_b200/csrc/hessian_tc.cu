@@ -78,7 +78,8 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -93,6 +94,7 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
       tc::mbar_init(acc_full + i, 1);
       tc::mbar_init(acc_empty + i, 8);
     }
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -104,6 +106,7 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  int64_t issued = 0;             // stages filled by the producer thread
 
   if (warp == 0) {
     if (lane == 0) {
@@ -124,6 +127,7 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
           for (int q = 0; q < BM / 64; ++q) tc::tma_load_2d(a + q * BOX_BYTES, &xmap, i0 + 64 * q, y, full + stage);
 #pragma unroll
           for (int q = 0; q < BN / 64; ++q) tc::tma_load_2d(b + q * BOX_BYTES, &xmap, j0 + 64 * q, y, full + stage);
+          ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
@@ -220,7 +224,19 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) raise_status(status, GPTQ_ERR_TIMEOUT);
+  if (*abort_flag) {
+    // A wait gave up (every role has left its loop, so the flag is final and the
+    // branch is uniform): the producer's copies and the issued MMAs land before
+    // TMEM is freed and the CTA exits.
+    if (warp == 0 && lane == 0) tc::drain_tma_ring(full, STAGES, issued);
+    if (warp == 1 && lane == 0) {
+      tc::mma_commit(drain);
+      tc::mbar_drain(drain, 0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0) raise_status(status, GPTQ_ERR_TIMEOUT);
+  }
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem_base, TMEM_COLS);

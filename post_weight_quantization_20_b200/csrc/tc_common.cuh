@@ -58,6 +58,28 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   return false;
 }
 
+// Bounded wait that does not stop at the abort flag.  After an abort, the thread
+// that issued TMA copies or MMAs waits with it until they have landed, so that
+// the CTA frees TMEM and exits with none of its own copies in flight.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity,
+                                           uint32_t limit = WAIT_LIMIT) {
+  for (uint32_t it = 0; it < limit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
+// Drain the TMA copies of a ring of `stages` full barriers, each filled once per
+// issue (one arrive.expect_tx and its copies) in round-robin order, after
+// `issued` issues in all: stage s was filled n_s times and its last phase has
+// parity (n_s - 1) & 1.  Earlier phases of a stage completed before it was
+// refilled, so only the last one of each stage can still be pending.
+__device__ __forceinline__ void drain_tma_ring(uint64_t* full, int stages, int64_t issued) {
+  for (int s = 0; s < stages; ++s) {
+    const int64_t n = issued / stages + (s < issued % stages ? 1 : 0);
+    if (n > 0) mbar_drain(full + s, uint32_t((n - 1) & 1));
+  }
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
   asm volatile(

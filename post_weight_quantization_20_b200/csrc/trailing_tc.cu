@@ -45,7 +45,8 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + BUFS * STAGE);
   uint64_t* empty = full + BUFS;
   uint64_t* done = empty + BUFS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* drain = done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * TM, n0 = e + blockIdx.x * TN;
@@ -56,6 +57,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
       tc::mbar_init(empty + b, 1);
     }
     tc::mbar_init(done, 1);
+    tc::mbar_init(drain, 1);
     *abort_flag = 0;
     tc::fence_barrier_init();
   }
@@ -67,6 +69,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
+  int64_t issued = 0;             // stages filled by the producer thread
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < nk; ++s) {
@@ -83,6 +86,7 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
         tc::tma_load_2d(bh + q * B_BOX, &uhi, i0 + k0, n0 + 128 * q, full + b);
         tc::tma_load_2d(bl + q * B_BOX, &ulo, i0 + k0, n0 + 128 * q, full + b);
       }
+      ++issued;
     }
   } else if (warp == 1 && lane == 0) {
     bool ok = true;
@@ -178,7 +182,18 @@ k_trailing_tc(const __grid_constant__ CUtensorMap ehi, const __grid_constant__ C
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (threadIdx.x == 0 && *abort_flag) raise_status(status, GPTQ_ERR_TIMEOUT);
+  if (*abort_flag) {
+    // A wait gave up (the flag is final here and the branch uniform): the
+    // producer's copies and the issued MMAs land before TMEM is freed.
+    if (warp == 0 && lane == 0) tc::drain_tma_ring(full, BUFS, issued);
+    if (warp == 1 && lane == 0) {
+      tc::mma_commit(drain);
+      tc::mbar_drain(drain, 0);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (threadIdx.x == 0) raise_status(status, GPTQ_ERR_TIMEOUT);
+  }
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, TN);
