@@ -36,11 +36,12 @@ from post_weight_quantization_20_b200.workloads import WORKLOADS  # noqa: E402
 
 METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per Hessian launch from the ncu capture summarised in
-# profiles/hessian_tc_C3072_T65536.md (C = 3072, 65536 tokens: 734.9 MB + 135.5 MB),
-# scaled to the bench's 262144-token launch by the token count.  Set to None when
-# the kernel changes until it is captured again.
-HESSIAN_TRAFFIC = {"bytes_per_token_C3072": (734.898432e6 + 135.484416e6) / 65536}
+# DRAM bytes (read + write) per Hessian launch from an ncu capture of the current
+# kernel (a small case scaled to the bench's launch by the token count), or None.
+# The capture summarised in profiles/hessian_tc_C3072_T65536.md (C = 3072, 65536
+# tokens: 734.9 MB + 135.5 MB) predates the kernel's abort-path drain, so the
+# figure stays None until the kernel is captured again.
+HESSIAN_TRAFFIC = None
 
 
 def load_peaks():
