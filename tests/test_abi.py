@@ -183,3 +183,24 @@ def test_binding_checks_buffer_shapes_before_calling_the_library():
         G.gptq_quantize_layer(torch.zeros(0, C, dtype=torch.float16), U, perm, cfg,
                               torch.zeros(0, dtype=torch.uint8), torch.zeros(0), torch.zeros(0),
                               ok["g_idx"], ok["losses"], ok["ws"])
+
+
+def test_header_compiles_as_c99_and_the_library_links(tmp_path):
+    # a plain C caller: no C++ in the header, the library links without torch, and the
+    # calls that need no device answer before anything is launched
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    G.load_library()                                  # builds nothing; the .so must exist
+    libdir = os.path.dirname(G.LIB_PATH)
+    exe = tmp_path / "c_abi_check"
+    src = os.path.join(ROOT, "tests", "c_abi_check.c")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic",
+                        "-I", os.path.join(ROOT, "include"), src, "-o", str(exe),
+                        "-L", libdir, "-lgptq", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
