@@ -204,3 +204,46 @@ def test_header_compiles_as_c99_and_the_library_links(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and "c abi ok" in r.stdout, r.stdout + r.stderr
+
+
+class _FakeLib:
+    """Stands in for libgptq: records the calls, returns GPTQ_OK, computes nothing."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        if not name.startswith("gptq_"):
+            raise AttributeError(name)
+
+        def call(*args):
+            self.calls.append(name)
+            if name == "gptq_workspace_size":
+                return 4096
+            if name == "gptq_hessian_accumulate":
+                n = args[1]._obj
+                n.value += int(args[4])
+            return 0
+        return call
+
+
+@pytest.mark.parametrize("rows,cols,group,act", [(8, 128, 128, False), (5, 96, 32, True),
+                                                  (3, 40, 0, False), (0, 64, 64, False)])
+def test_layer_helpers_pass_the_buffer_checks(monkeypatch, rows, cols, group, act):
+    # the one-layer helpers allocate every buffer themselves; with the device and the
+    # library faked out on CPU, every buffer they pass must satisfy the wrappers' checks
+    fake = _FakeLib()
+    monkeypatch.setattr(G, "load_library", lambda *a: fake)
+    monkeypatch.setattr(G, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(G, "_stream", lambda s: None)
+    cfg = G.make_config(4, group, act_order=act)
+    W = torch.zeros(rows, cols, dtype=torch.float16)
+    X = torch.zeros(50, cols, dtype=torch.float16)
+    r = G.quantize_layer(W, X, cfg, chunk_tokens=20)
+    assert r.n_tokens == 50 and r.packed.shape == (rows, G.packed_words(cols, 4))
+    assert fake.calls.count("gptq_hessian_accumulate") == 3
+    assert fake.calls[-2:] == ["gptq_quantize_layer", "gptq_pack"]
+    shared = G.quantize_layers_shared([W, torch.zeros(rows + 2, cols, dtype=torch.bfloat16)], X, cfg)
+    assert [x.codes.shape for x in shared] == [(rows, cols), (rows + 2, cols)]
+    rtn = G.quantize_rtn(W, cfg)
+    assert rtn.scales.shape == (rows, G.n_groups(cols, group))
