@@ -473,3 +473,14 @@ def test_dequant_matmul_one_hot_inputs_pick_weight_columns():
     Y = o.dequant_matmul(np.eye(16), o.pack(out["codes"], 3), out["scales"], out["zeros"],
                          out["g_idx"], 3)
     np.testing.assert_array_equal(Y, out["Q"].T)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_packing_density_matches_the_quoted_model_sizes(bits):
+    """A 175B-parameter model takes ~87.5 GB at 4 bits and ~65.6 GB at 3 bits
+    ([Deep-dive §4.3]), i.e. exactly bits/8 bytes per weight: at the OPT-175B layer
+    widths (12288, 49152 columns) the packed rows carry no padding."""
+    for cols in (12288, 49152):
+        codes = np.zeros((2, cols), dtype=np.int64)
+        assert o.pack(codes, bits).nbytes == 2 * cols * bits // 8
+    assert 175e9 * bits / 8 / 1e9 == pytest.approx({4: 87.5, 3: 65.6}[bits], abs=0.05)
