@@ -347,7 +347,10 @@ def run_ours(args, rank, world, local_rank):
             outs.append(r)
         return outs
 
-    e2e_step()
+    # two untimed steps: each step's pinned outputs stay alive while the next one
+    # runs, so the caching host allocator holds two sets before the timed region
+    outs = e2e_step()
+    outs = e2e_step()
     torch.cuda.synchronize(dev)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)

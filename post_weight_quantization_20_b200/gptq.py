@@ -429,7 +429,6 @@ class HostResult:
 
 
 _copy_streams: dict = {}
-_pinned_cache: dict = {}
 
 
 def _side_stream(dev) -> torch.cuda.Stream:
@@ -439,22 +438,18 @@ def _side_stream(dev) -> torch.cuda.Stream:
     return _copy_streams[key]
 
 
-def _pinned(key, shape, dtype) -> torch.Tensor:
-    k = (key, tuple(shape), dtype)
-    if k not in _pinned_cache:
-        _pinned_cache[k] = torch.empty(shape, dtype=dtype, pin_memory=True)
-    return _pinned_cache[k]
-
-
 def quantize_layer_host(W_host: torch.Tensor, X_host: torch.Tensor, cfg: gptq_config, device=None,
-                        chunk_tokens: int = 32768, stream=None, tag: str = "") -> HostResult:
+                        chunk_tokens: int = 32768, stream=None) -> HostResult:
     """Quantize one layer whose W and X live in pinned host memory.
 
     X is uploaded in chunks on a side stream while the previous chunk is being
     accumulated into H on the compute stream (two device staging buffers); the
     packed codes, scales, zeros, g_idx, losses and perm are copied back into
     pinned host tensors.  Asynchronous: synchronize the stream before reading
-    the result (result.status holds the device status word).
+    the result (result.status holds the device status word).  Every call returns
+    its own pinned tensors (torch's caching host allocator hands a freed block out
+    again only after the copies into it have completed), so results of several
+    layers in flight never share memory.
     """
     dev = torch.device(device) if device is not None else torch.device("cuda")
     comp = stream if stream is not None else torch.cuda.current_stream(dev)
@@ -505,8 +500,8 @@ def quantize_layer_host(W_host: torch.Tensor, X_host: torch.Tensor, cfg: gptq_co
         gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, wsq, status, comp)
         packed = torch.empty(R, packed_words(C, cfg.bits), dtype=torch.int32, device=dev)
         gptq_pack(codes, cfg.bits, packed, comp)
-        host = HostResult(*(_pinned((tag, i), t.shape, t.dtype) for i, t in
-                            enumerate((packed, scales, zeros, g_idx, losses, perm, status))))
+        host = HostResult(*(torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in
+                            (packed, scales, zeros, g_idx, losses, perm, status)))
         for dst, src in zip((host.packed, host.scales, host.zeros, host.g_idx, host.losses,
                              host.perm, host.status),
                             (packed, scales, zeros, g_idx, losses, perm, status)):
