@@ -396,8 +396,10 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "traffic_scope": "bytes per C=3072 launch (the largest Hessian of the "
-                                      "workload), ncu capture at 65536 tokens scaled by tokens",
+                     "traffic_scope": ("bytes per C=3072 launch (the largest Hessian of the "
+                                       "workload), ncu capture at 65536 tokens scaled by tokens")
+                     if traffic is not None else
+                     "null: the kernel changed after its last ncu capture",
                      "peak_source": f"{peaks['source']} bf16 dense burst"},
         "e2e": {"value": e2e_ms / len(layers), "unit": "ms", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
