@@ -288,13 +288,18 @@ def run_ours(args, rank, world, local_rank):
         if world > 1:
             dist.barrier()
 
+    def check_status(where):
+        # a device condition (a bounded wait that gave up, a non-PD pivot) makes the
+        # kernels finish early, so the run's times would not be of the whole work
+        for b in layers:
+            st = int(b["status"].item())
+            if st:
+                raise RuntimeError(f"device status {G.status_names(st)} {where}")
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-    for b in layers:
-        st = int(b["status"].item())
-        if st:
-            raise RuntimeError(f"device status {G.status_names(st)}")
+    check_status("after the warm-up steps")
 
     clocks = ClockSampler(dev)
     barrier()
@@ -311,6 +316,7 @@ def run_ours(args, rank, world, local_rank):
     launches = G.gptq_launch_count() - launches0
     barrier()
     cl = clocks.stop()
+    check_status("in the timed steps")
     ms = t0.elapsed_time(t1)
     hess_ms = sum(a.elapsed_time(b) for a, b, _, _ in hess_ev)
     # per phase, summed over the layers of one step, and each phase's useful
