@@ -290,11 +290,17 @@ def run_ours(args, rank, world, local_rank):
 
     def check_status(where):
         # a device condition (a bounded wait that gave up, a non-PD pivot) makes the
-        # kernels finish early, so the run's times would not be of the whole work
+        # kernels finish early, so the run's times would not be of the whole work;
+        # every rank takes the same collective here and raises together
+        st = 0
         for b in layers:
-            st = int(b["status"].item())
-            if st:
-                raise RuntimeError(f"device status {G.status_names(st)} {where}")
+            st |= int(b["status"].item())
+        if world > 1:
+            t = torch.tensor([st], dtype=torch.int64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            st = st or int(t.item())
+        if st:
+            raise RuntimeError(f"device status {G.status_names(st)} {where}")
 
     for _ in range(args.warmup):
         step()
