@@ -21,6 +21,7 @@ void note_error(cudaError_t e, const char* where) {
 
 using namespace gptq;
 
+
 static bool valid_dtype(int dt) { return dt == GPTQ_F32 || dt == GPTQ_F16 || dt == GPTQ_BF16; }
 
 static gptq_status check_cfg(const gptq_config* cfg) {
@@ -60,6 +61,7 @@ size_t gptq_workspace_size(int op, int64_t rows, int64_t cols, const gptq_config
 gptq_status gptq_hessian_accumulate(float* H, int64_t* n_seen, const void* X, int xdtype,
                                     int64_t m_tokens, int64_t cols, int64_t ldx,
                                     int32_t* dev_status, void* stream) {
+  CallRange range_("gptq_hessian_accumulate");
   if (!H || !n_seen || cols <= 0 || cols > INT_MAX / 2 || m_tokens < 0 || *n_seen < 0)
     return GPTQ_ERR_INVALID_ARG;
   if (!valid_dtype(xdtype) || ldx < cols) return GPTQ_ERR_INVALID_ARG;
@@ -81,6 +83,7 @@ gptq_status gptq_hessian_accumulate(float* H, int64_t* n_seen, const void* X, in
 gptq_status gptq_prepare(const float* H, int64_t cols, const gptq_config* cfg, float* U,
                          int32_t* perm, void* ws, size_t ws_bytes, int32_t* dev_status,
                          void* stream) {
+  CallRange range_("gptq_prepare");
   if (!H || !U || !perm || cols <= 0 || cols > INT_MAX / 2) return GPTQ_ERR_INVALID_ARG;
   GPTQ_TRY(check_cfg(cfg));
   if (!ws || !aligned256(ws)) return GPTQ_ERR_INVALID_ARG;
@@ -93,6 +96,7 @@ gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t
                                 const gptq_config* cfg, uint8_t* codes, float* scales,
                                 float* zeros, int32_t* g_idx, float* losses, void* ws,
                                 size_t ws_bytes, int32_t* dev_status, void* stream) {
+  CallRange range_("gptq_quantize_layer");
   if (cols <= 0 || cols > INT_MAX / 2 || rows < 0 || rows > INT_MAX) return GPTQ_ERR_INVALID_ARG;
   if (!U || !perm || !g_idx || !losses) return GPTQ_ERR_INVALID_ARG;
   if (rows > 0 && (!W || !codes || !scales || !zeros)) return GPTQ_ERR_INVALID_ARG;
@@ -107,6 +111,7 @@ gptq_status gptq_quantize_layer(const void* W, int wdtype, int64_t rows, int64_t
 
 gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits,
                       uint32_t* packed, void* stream) {
+  CallRange range_("gptq_pack");
   if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0) return GPTQ_ERR_INVALID_ARG;
   if (rows > 0 && cols > 0 && (!codes || !packed)) return GPTQ_ERR_INVALID_ARG;
@@ -128,6 +133,7 @@ const char* gptq_status_string(int status) {
 }
 
 gptq_status gptq_selftest_timeout(int which, int32_t* dev_status, void* stream) {
+  CallRange range_("gptq_selftest_timeout");
   if (!dev_status) return GPTQ_ERR_INVALID_ARG;
   if (which == GPTQ_SELFTEST_MBARRIER) return selftest_mbarrier(as_stream(stream), dev_status);
   if (which == GPTQ_SELFTEST_GRID_BARRIER)

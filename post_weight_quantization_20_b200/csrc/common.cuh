@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "gptq.h"
@@ -26,6 +27,16 @@ __device__ __forceinline__ float load_f32(const void* p, int dt, int64_t idx) {
   if (dt == GPTQ_F16) return __half2float(static_cast<const __half*>(p)[idx]);
   return __bfloat162float(static_cast<const __nv_bfloat16*>(p)[idx]);
 }
+
+// An NVTX range around one ABI call, so that a profiler can select a call's
+// kernels (e.g. ncu --nvtx --nvtx-include "gptq_prepare/"); without a tool
+// attached the push and pop return at once.
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+  CallRange(const CallRange&) = delete;
+  CallRange& operator=(const CallRange&) = delete;
+};
 
 // Opt a kernel into more than 48 KB of dynamic shared memory (idempotent).
 template <typename K>

@@ -50,6 +50,7 @@ using namespace gptq;
 extern "C" gptq_status gptq_prepare_static(const float* H, int64_t cols, const gptq_config* cfg,
                                            float* U, int32_t* perm, int32_t* dev_status,
                                            void* stream) {
+  gptq::CallRange range_("gptq_prepare_static");
   if (!H || !U || !perm || cols <= 0 || !cfg) return GPTQ_ERR_INVALID_ARG;
   if (cfg->bits != 2 && cfg->bits != 3 && cfg->bits != 4 && cfg->bits != 8)
     return GPTQ_ERR_INVALID_ARG;
