@@ -296,6 +296,7 @@ class LayerResult:
     H: torch.Tensor
     U: torch.Tensor
     n_tokens: int
+    damp: float | None = None      # the relative damping the factor was formed with
 
 
 def check_status(status: torch.Tensor, where: str = "device") -> None:
@@ -333,6 +334,29 @@ def _factor(H, cfg, perm, rows, dev, status, stream):
     return U, perm
 
 
+def _with_damp(cfg: gptq_config, damp: float) -> gptq_config:
+    return gptq_config(cfg.bits, cfg.group_size, cfg.sym, cfg.act_order, float(damp),
+                       cfg.block_size)
+
+
+def _factor_retry(H, cfg, perm, rows, dev, status, stream, damp_retry):
+    """Factor H; while the factorization reports a non-positive pivot (and nothing
+    else) and larger damping values remain in `damp_retry`, factor again with the
+    next one.  A near-singular Hessian from a small calibration set is stabilised
+    by a larger damp_percent, e.g. 0.1 (GPTQ量化算法深度解析 §3.3).  Without retry
+    values nothing is synchronised.  Returns (U, perm, the damp used)."""
+    U, p = _factor(H, cfg, perm, rows, dev, status, stream)
+    damp = float(cfg.damp)
+    for d in damp_retry:
+        code = int(status.item())
+        if code != GPTQ_ERR_NOT_PD:
+            break
+        status.zero_()
+        U, p = _factor(H, _with_damp(cfg, d), perm, rows, dev, status, stream)
+        damp = float(d)
+    return U, p, damp
+
+
 def _sweep(W, U, perm, cfg, dev, status, stream):
     R, C = W.shape
     G = n_groups(C, cfg.group_size)
@@ -349,24 +373,27 @@ def _sweep(W, U, perm, cfg, dev, status, stream):
 
 
 def quantize_layer(W: torch.Tensor, X, cfg: gptq_config, perm: torch.Tensor | None = None,
-                   chunk_tokens: int | None = None, stream=None, check: bool = True) -> LayerResult:
+                   chunk_tokens: int | None = None, stream=None, check: bool = True,
+                   damp_retry=()) -> LayerResult:
     """Quantize one linear layer.  W (rows x cols) and X (tokens x cols, or an
-    iterable of such chunks) are device tensors."""
+    iterable of such chunks) are device tensors.  damp_retry: larger relative
+    damping values to factor with, in turn, while the factorization reports a
+    non-positive pivot (e.g. (0.1,)); each retry synchronises the stream once."""
     dev = W.device
     R, C = W.shape
     with _on(stream):
         status = torch.zeros(1, dtype=torch.int32, device=dev)
         H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
-        U, perm = _factor(H, cfg, perm, R, dev, status, stream)
+        U, perm, damp = _factor_retry(H, cfg, perm, R, dev, status, stream, damp_retry)
         codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status, stream)
     if check:
         check_status(status, "quantize_layer")
-    return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n)
+    return LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n, damp)
 
 
 def quantize_layers_shared(Ws, X, cfg: gptq_config, perm: torch.Tensor | None = None,
                            chunk_tokens: int | None = None, stream=None,
-                           check: bool = True) -> list:
+                           check: bool = True, damp_retry=()) -> list:
     """Quantize several linear layers that read the same input (the q/k/v or
     gate/up projections of one block): one Hessian and one factorization, then one
     sweep per weight.  Each W is rows_i x cols; the results are those of separate
@@ -382,11 +409,13 @@ def quantize_layers_shared(Ws, X, cfg: gptq_config, perm: torch.Tensor | None = 
     with _on(stream):
         status = torch.zeros(1, dtype=torch.int32, device=dev)
         H, n = _hessian(X, C, dev, status, chunk_tokens, stream)
-        U, perm = _factor(H, cfg, perm, max(W.shape[0] for W in Ws), dev, status, stream)
+        U, perm, damp = _factor_retry(H, cfg, perm, max(W.shape[0] for W in Ws), dev, status,
+                                      stream, damp_retry)
         for W in Ws:
             codes, scales, zeros, g_idx, losses, packed = _sweep(W, U, perm, cfg, dev, status,
                                                                  stream)
-            out.append(LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n))
+            out.append(LayerResult(codes, scales, zeros, g_idx, losses, perm, packed, H, U, n,
+                                   damp))
     if check:
         check_status(status, "quantize_layers_shared")
     return out

@@ -247,3 +247,63 @@ def test_layer_helpers_pass_the_buffer_checks(monkeypatch, rows, cols, group, ac
     assert [x.codes.shape for x in shared] == [(rows, cols), (rows + 2, cols)]
     rtn = G.quantize_rtn(W, cfg)
     assert rtn.scales.shape == (rows, G.n_groups(cols, group))
+
+
+class _PivotFakeLib(_FakeLib):
+    """gptq_prepare reports a non-positive pivot while damp < `needs`; the Hessian can
+    report non-finite data instead."""
+
+    def __init__(self, needs, nonfinite=False):
+        super().__init__()
+        self.needs, self.nonfinite, self.damps = needs, nonfinite, []
+
+    def __getattr__(self, name):
+        base = super().__getattr__(name)
+        if name not in ("gptq_prepare", "gptq_hessian_accumulate"):
+            return base
+
+        def call(*args):
+            r = base(*args)
+            if name == "gptq_prepare":
+                damp = args[2]._obj.damp
+                self.damps.append(round(damp, 6))
+                if damp < self.needs:
+                    ctypes.c_int32.from_address(args[7].value).value |= G.GPTQ_ERR_NOT_PD
+            elif self.nonfinite:
+                ctypes.c_int32.from_address(args[7].value).value |= G.GPTQ_ERR_NONFINITE
+            return r
+        return call
+
+
+def _run_retry(monkeypatch, fake, **kw):
+    monkeypatch.setattr(G, "load_library", lambda *a: fake)
+    monkeypatch.setattr(G, "_need_cuda", lambda *ts: None)
+    monkeypatch.setattr(G, "_stream", lambda s: None)
+    W = torch.zeros(4, 64, dtype=torch.float16)
+    X = torch.zeros(10, 64, dtype=torch.float16)
+    return G.quantize_layer(W, X, G.make_config(4, 64, damp=0.01), **kw)
+
+
+def test_damping_retry_refactors_until_the_pivots_are_positive(monkeypatch):
+    # a near-singular Hessian is stabilised by a larger damp_percent (e.g. 0.1)
+    fake = _PivotFakeLib(needs=0.1)
+    r = _run_retry(monkeypatch, fake, damp_retry=(0.05, 0.1, 0.5))
+    assert fake.damps == [0.01, 0.05, 0.1] and r.damp == pytest.approx(0.1)
+    fake = _PivotFakeLib(needs=0.0)                       # no retry needed
+    r = _run_retry(monkeypatch, fake, damp_retry=(0.1,))
+    assert fake.damps == [0.01] and r.damp == pytest.approx(0.01)
+
+
+def test_damping_retry_gives_up_and_leaves_other_conditions_alone(monkeypatch):
+    fake = _PivotFakeLib(needs=1.0)                       # every value too small
+    with pytest.raises(G.GPTQError) as e:
+        _run_retry(monkeypatch, fake, damp_retry=(0.1,))
+    assert e.value.code == G.GPTQ_ERR_NOT_PD and fake.damps == [0.01, 0.1]
+    fake = _PivotFakeLib(needs=0.1)                       # no retry values: no retry
+    with pytest.raises(G.GPTQError):
+        _run_retry(monkeypatch, fake)
+    assert fake.damps == [0.01]
+    fake = _PivotFakeLib(needs=0.1, nonfinite=True)       # non-finite data is not retried
+    with pytest.raises(G.GPTQError) as e:
+        _run_retry(monkeypatch, fake, damp_retry=(0.1,))
+    assert e.value.code & G.GPTQ_ERR_NONFINITE and fake.damps == [0.01]
