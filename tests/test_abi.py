@@ -307,3 +307,18 @@ def test_damping_retry_gives_up_and_leaves_other_conditions_alone(monkeypatch):
     with pytest.raises(G.GPTQError) as e:
         _run_retry(monkeypatch, fake, damp_retry=(0.1,))
     assert e.value.code & G.GPTQ_ERR_NONFINITE and fake.damps == [0.01]
+
+
+def test_guarded_buffers_detect_writes_past_either_end():
+    # the helper the GPU canary test uses, checked on CPU
+    from tests.guards import MARGIN, Guarded
+    g = Guarded((3, 5), torch.float32, "cpu")
+    assert g.t.is_contiguous() and g.t.data_ptr() % 256 == g.raw.data_ptr() % 256
+    g.t.fill_(1.0)                                     # writes inside the view only
+    assert g.intact()
+    g.raw[MARGIN + g.nbytes] = 0                       # one byte past the end
+    assert not g.intact()
+    h = Guarded((7,), torch.uint8, "cpu", fill=torch.arange(7, dtype=torch.uint8))
+    assert h.t.tolist() == list(range(7)) and h.intact()
+    h.raw[MARGIN - 1] = 1                              # one byte before the start
+    assert not h.intact()
