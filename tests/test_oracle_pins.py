@@ -484,3 +484,4 @@ def test_packing_density_matches_the_quoted_model_sizes(bits):
         codes = np.zeros((2, cols), dtype=np.int64)
         assert o.pack(codes, bits).nbytes == 2 * cols * bits // 8
     assert 175e9 * bits / 8 / 1e9 == pytest.approx({4: 87.5, 3: 65.6}[bits], abs=0.05)
+
