@@ -1,7 +1,7 @@
 """Guarded buffers for the library's outputs: every buffer is a view into a larger
 byte buffer whose margins hold a fixed pattern, so that a write past either end of
-the view shows up as a changed margin byte (SURVEY-listed stand-in for a memory
-checker, which is not available on the test machines)."""
+the view shows up as a changed margin byte (a check of out-of-bounds writes that
+needs no memory-checking tool)."""
 import torch
 
 MARGIN = 4096          # bytes on each side; keeps 256-byte alignment of the view
