@@ -1,7 +1,7 @@
 """The multi-GPU layer path (sharded.py) as gloo ranks on CPU.
 
-Calibration tokens are split unevenly over two ranks (one case gives a rank no
-tokens) and the rows of W are split by row_range.  The library's three steps are
+Calibration tokens are split unevenly over two or three ranks (some cases give a
+rank no tokens) and the rows of W are split by row_range.  The library's three steps are
 replaced on CPU by stand-ins: the Hessian of the rank's tokens in torch, and the
 oracle's factorization and sweep.  What is checked is the sharding itself:
   * the combined H equals the Hessian of all tokens and is bitwise the same on
@@ -67,7 +67,7 @@ def _cpu_steps(G, o):
     return hessian, factor, sweep
 
 
-def _rank(rank, world, port, split, q):
+def _rank(rank, world, port, split, qcfg, q):
     import datetime
 
     import torch.distributed as dist
@@ -88,7 +88,8 @@ def _rank(rank, world, port, split, q):
         W = (0.02 * rng.standard_normal((R, C))).astype(np.float32)
         t0 = sum(split[:rank])
         r0, r1 = SH.row_range(R, world, rank)
-        cfg = G.make_config(4, 16, act_order=True)
+        bits, group, act = qcfg
+        cfg = G.make_config(bits, group, act_order=act)
         res = SH.quantize_layer_sharded(torch.from_numpy(W[r0:r1]),
                                         torch.from_numpy(X[t0:t0 + split[rank]]), cfg,
                                         check=False)
@@ -100,13 +101,16 @@ def _rank(rank, world, port, split, q):
 
 
 @pytest.mark.timeout(180)
-@pytest.mark.parametrize("split", [(700, 300), (1000, 0)])
-def test_two_ranks_shard_tokens_and_rows(split):
+@pytest.mark.parametrize("split,qcfg", [((700, 300), (4, 16, True)), ((1000, 0), (4, 16, True)),
+                                        ((500, 0, 300), (3, 0, False))],
+                         ids=["2-ranks", "2-ranks-one-empty", "3-ranks-per-row"])
+def test_ranks_shard_tokens_and_rows(split, qcfg):
     from oracle import gptq_ref as o
-    world, port = 2, _free_port()
+    world, port = len(split), _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, split, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, split, qcfg, q))
+             for r in range(world)]
     for p in procs:
         p.start()
     out = sorted((q.get(timeout=150) for _ in range(world)), key=lambda t: t[0])
@@ -118,15 +122,16 @@ def test_two_ranks_shard_tokens_and_rows(split):
     X = (rng.standard_normal((sum(split), C)) @ rng.standard_normal((C, C)) * 0.3).astype(np.float32)
     W = (0.02 * rng.standard_normal((R, C))).astype(np.float32)
     H_all, n = o.hessian(X.astype(np.float64))
-    H0, H1 = out[0][4], out[1][4]
-    assert np.array_equal(H0, H1)                        # every rank factors the same bits
+    H0 = out[0][4]
+    assert all(np.array_equal(H0, t[4]) for t in out)   # every rank factors the same bits
     assert np.linalg.norm(H0 - H_all) <= 1e-6 * np.linalg.norm(H_all)
     assert all(t[3] == n for t in out)
     # the full layer on the same H: each rank holds exactly its rows
     # the ranks' config holds damp as a float32 (0.00999999977...), as the C struct does
-    p, _, U = o.prepare(H0.astype(np.float64), float(np.float32(0.01)), True)
+    bits, group, act = qcfg
+    p, _, U = o.prepare(H0.astype(np.float64), float(np.float32(0.01)), act)
     U = U.astype(np.float32).astype(np.float64)
-    full = o.finalize(o.sweep(W.astype(np.float64)[:, p], U, 4, 16, False, 128), p, 16)
+    full = o.finalize(o.sweep(W.astype(np.float64)[:, p], U, bits, group, False, 128), p, group)
     for rank, r0, r1, _, _, codes, scales, zeros, losses in out:
         np.testing.assert_array_equal(codes, full["codes"][r0:r1])
         np.testing.assert_array_equal(scales, full["scales"][r0:r1].astype(np.float32))
