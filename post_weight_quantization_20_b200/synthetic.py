@@ -129,8 +129,14 @@ def outlier_channels(cols: int, spec: ActSpec, seed: int, tag: int) -> np.ndarra
 
 
 def gen_activations(tokens: int, cols: int, dtype: str, spec: ActSpec, seed: int,
-                    tag: int = 0, threads: int | None = None) -> np.ndarray:
-    """X (tokens x cols) in storage format ``dtype``, generated in CHUNK-token pieces."""
+                    tag: int = 0, threads: int | None = None, first_token: int = 0) -> np.ndarray:
+    """X (tokens x cols) in storage format ``dtype``, generated in CHUNK-token pieces.
+    ``first_token`` (a multiple of CHUNK) starts the block further into the same
+    stream, so a large calibration set can be produced piece by piece: the rows
+    equal those of one call that covers them all."""
+    if first_token < 0 or first_token % CHUNK:
+        raise ValueError(f"first_token must be a non-negative multiple of {CHUNK}")
+    k0 = first_token // CHUNK
     threads = _threads() if threads is None else threads
     chan = np.ones(cols, dtype=np.float32)
     idx = outlier_channels(cols, spec, seed, tag)
@@ -147,7 +153,7 @@ def gen_activations(tokens: int, cols: int, dtype: str, spec: ActSpec, seed: int
     def work(k):
         t0 = starts[k]
         m = min(CHUNK, tokens - t0)
-        g = _rng(seed, tag, k)
+        g = _rng(seed, tag, k0 + k)
         if spec.dist == "t4":
             a = _student_t4(g, m * cols).reshape(m, cols)
         elif spec.dist == "normal":

@@ -79,3 +79,13 @@ def test_to_f64_is_exact_widening(dtype):
     x64 = S.to_f64(X, dtype)
     x32 = S.to_f32(X, dtype)
     assert x64.dtype == np.float64 and np.array_equal(x64, x32.astype(np.float64))
+
+
+def test_a_token_range_equals_the_same_rows_of_one_call():
+    spec = S.ActSpec(mix_rank=2)
+    whole = S.gen_activations(3 * S.CHUNK + 17, 24, S.F16, spec, seed=3, tag=4)
+    part = S.gen_activations(S.CHUNK + 17, 24, S.F16, spec, seed=3, tag=4,
+                             first_token=2 * S.CHUNK)
+    assert np.array_equal(part.view(np.uint16), whole[2 * S.CHUNK:].view(np.uint16))
+    with pytest.raises(ValueError):
+        S.gen_activations(10, 24, S.F16, spec, seed=3, first_token=5)
