@@ -26,6 +26,10 @@
  *    caller reads *dev_status after synchronizing the stream.
  *  - Matrices are row-major.  W is rows x cols (out x in features, as a PyTorch
  *    Linear weight); X is tokens x cols.
+ *  - Host threads: the calls may be made from several host threads at once.  The
+ *    side stream of gptq_quantize_layer and the text of gptq_last_error are kept
+ *    per host thread, and the launch counter is atomic; gptq_prepare_static is the
+ *    one call whose scratch memory is shared (see there).
  */
 #ifndef GPTQ_H_
 #define GPTQ_H_
