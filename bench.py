@@ -208,6 +208,18 @@ def max_over_ranks(vals, world, device):
     return [float(v) for v in t.tolist()]
 
 
+def status_over_ranks(local_status, world, device):
+    """A device status word that is nonzero on any rank, on every rank (every rank
+    takes this collective, so all of them raise together on an error)."""
+    if world == 1:
+        return int(local_status)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([int(local_status)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return int(local_status) or int(t.item())
+
+
 def job_ms_per_layer(ms_timed, steps, layers_per_rank, world):
     """Whole-job ms per layer: every rank quantizes `layers_per_rank` layers per step
     (replicas, weak scaling), all finished within the slowest rank's time."""
@@ -295,10 +307,7 @@ def run_ours(args, rank, world, local_rank):
         st = 0
         for b in layers:
             st |= int(b["status"].item())
-        if world > 1:
-            t = torch.tensor([st], dtype=torch.int64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            st = st or int(t.item())
+        st = status_over_ranks(st, world, dev)
         if st:
             raise RuntimeError(f"device status {G.status_names(st)} {where}")
 

@@ -27,8 +27,11 @@ def _rank(rank, world, port, q):
         # rank 1 is the slow one for the first entry, rank 0 for the second
         got = bench.max_over_ranks([10.0 + rank, 7.0 - rank], world, "cpu")
         value = bench.job_ms_per_layer(got[0], 5, 3, world)
+        # a device condition on rank 1 only: both ranks see it and raise together
+        st = bench.status_over_ranks(8 if rank == 1 else 0, world, "cpu")
+        clean = bench.status_over_ranks(0, world, "cpu")
         dist.barrier()
-        q.put((rank, got, value))
+        q.put((rank, got, value, st, clean))
     finally:
         dist.destroy_process_group()
 
@@ -45,9 +48,10 @@ def test_two_gloo_ranks_reduce_like_the_benchmark():
     for p in procs:
         p.join(timeout=30)
         assert p.exitcode == 0
-    for rank, got, value in out:
+    for rank, got, value, st, clean in out:
         assert got == [11.0, 7.0]                 # the max over ranks, on every rank
         assert value == pytest.approx(11.0 / 5 / (3 * world))
+        assert st != 0 and clean == 0
 
 
 def test_single_rank_needs_no_process_group():
