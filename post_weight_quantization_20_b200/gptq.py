@@ -397,7 +397,7 @@ def quantize_layers_shared(Ws, X, cfg: gptq_config, perm: torch.Tensor | None = 
     """Quantize several linear layers that read the same input (the q/k/v or
     gate/up projections of one block): one Hessian and one factorization, then one
     sweep per weight.  Each W is rows_i x cols; the results are those of separate
-    quantize_layer calls on the same X."""
+    quantize_layer calls on the same X.  damp_retry as for quantize_layer."""
     Ws = list(Ws)
     if not Ws:
         return []
