@@ -99,9 +99,12 @@ def hessian(X: np.ndarray, chunk: int | None = None):
 #         [Deep-dive §3.1 step 2], [Deep-dive §2.4], [Deep-dive §3.3]
 # -----------------------------------------------------------------------------
 def damp(H: np.ndarray, rel: float) -> np.ndarray:
-    """H + lambda I with lambda = rel * mean(diag H)."""
+    """H + lambda I with lambda = rel * mean(diag H) (a new array; lambda is added to
+    the diagonal entries only, which is H + lambda I entry for entry)."""
     lam = rel * float(np.mean(np.diag(H))) if H.shape[0] else 0.0
-    return H + lam * np.eye(H.shape[0])
+    Hd = np.array(H, dtype=np.float64, copy=True)
+    Hd[np.diag_indices(H.shape[0])] += lam
+    return Hd
 
 
 def act_order_perm(H: np.ndarray) -> np.ndarray:
@@ -112,8 +115,10 @@ def act_order_perm(H: np.ndarray) -> np.ndarray:
 def inverse_cholesky_upper(Hp: np.ndarray) -> np.ndarray:
     """U upper triangular with positive diagonal and U^T U = Hp^-1.
 
-    Textbook route: invert Hp through its Cholesky factorization, then take the
-    upper Cholesky factor of the inverse.
+    Textbook route: invert Hp through its Cholesky factorization Hp = L L^T
+    (LAPACK potri forms the lower triangle of Hp^-1 = L^-T L^-1 from L), then take
+    the upper Cholesky factor of the inverse (its lower triangle is all the
+    factorization reads).
     """
     C = Hp.shape[0]
     if C == 0:
@@ -122,12 +127,15 @@ def inverse_cholesky_upper(Hp: np.ndarray) -> np.ndarray:
         cf = sla.cho_factor(Hp, lower=True, check_finite=True)
     except (np.linalg.LinAlgError, ValueError) as e:
         raise NotPositiveDefinite(str(e)) from e
-    Hinv = sla.cho_solve(cf, np.eye(C))
-    Hinv = 0.5 * (Hinv + Hinv.T)
+    Hinv, info = sla.lapack.dpotri(cf[0], lower=1, overwrite_c=1)
+    del cf
+    if info != 0:
+        raise NotPositiveDefinite(f"potri info {info}")
     try:
         L = np.linalg.cholesky(Hinv)
     except np.linalg.LinAlgError as e:
         raise NotPositiveDefinite(str(e)) from e
+    del Hinv
     return L.T.copy()
 
 
@@ -139,6 +147,7 @@ def prepare(H: np.ndarray, rel_damp: float, act_order: bool, perm=None):
         perm = act_order_perm(H) if act_order else np.arange(C, dtype=np.int64)
     perm = np.asarray(perm, dtype=np.int64)
     Hp = Hd[np.ix_(perm, perm)]
+    del Hd
     U = inverse_cholesky_upper(Hp)
     return perm, Hp, U
 
