@@ -28,3 +28,17 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print every GPU-vs-oracle layer comparison (mismatches before and after the
+    near-tie replay, forced decisions and their largest distance from a tie, scale
+    and loss differences), so that the achieved tolerances are on record even in
+    a quiet run."""
+    mod = sys.modules.get("tests.parity")
+    lines = getattr(mod, "REPORT", None) if mod is not None else None
+    if not lines:
+        return
+    terminalreporter.write_sep("-", "parity against the float64 oracle")
+    for line in lines:
+        terminalreporter.write_line(line)

@@ -5,10 +5,10 @@ Bars (written in each test):
   * Hessian: relative Frobenius error of the upper triangle <= 1e-5 (fp32 accumulation);
   * inverse Cholesky factor: relative Frobenius error <= 1e-3 against the oracle's
     factor of the same (float32-rounded) Hessian;
-  * layer: after the near-tie replay (tests/parity.py) every code matches, forced
-    entries <= 0.1% of all codes and each within TAU grid steps of a tie, scales
-    within 1e-5 relative (within 1e-4 for group grids after forced upstream decisions),
-    zeros equal, reconstruction error ||(W - Q) X^T||^2 within 0.5%.
+  * layer (the stated tolerances, tests/parity.py): after the near-tie replay every
+    code matches, forced entries <= 0.1% of all codes and each within 1e-6 grid
+    steps of a midpoint, scales within 1e-5 relative, zeros equal, reconstruction
+    error ||(W - Q) X^T||^2 within 0.5%, per-column losses within 1e-3 (L1).
 """
 import numpy as np
 import pytest
@@ -21,7 +21,6 @@ from tests.parity import compare_layer
 
 pytestmark = pytest.mark.gpu
 
-TAU = 2e-3          # grid steps: fp32 state vs fp64 state (see design notes)
 DEV = "cuda"
 
 
@@ -214,15 +213,14 @@ def test_layer_parity(case):
     X = S.gen_activations(T, C, xdt, xspec, seed=R * 3 + C)
     out, H64, n = run_layer(W, wdt, X, xdt, bits, group, sym, act)
     W64 = S.to_f64(W, wdt)
-    p, ref = compare_layer(W64, H64, n, out["perm"], out, bits, group, sym, TAU)
+    p, ref = compare_layer(W64, H64, n, out["perm"], out, bits, group, sym)
     print(name, p.summary())
-    assert p.bad_hints == 0
-    assert p.code_mismatch == 0
-    assert p.forced_frac <= 1e-3
-    assert p.zero_diff == 0.0
-    assert p.scale_rel <= (1e-5 if group == 0 else 1e-4)
-    assert p.recon_rel <= 5e-3
-    assert p.loss_rel <= 1e-3
+    # a single column: every weight is an end point of its own row's grid, so the
+    # exact loss is rounding noise; there the losses are held to an absolute bar
+    # (1e-6 of the loss of quantizing every weight to zero) instead of a relative one
+    p.assert_bars(f"layer {name}", check_losses=(C > 1))
+    if C == 1:
+        assert p.loss_abs <= 1e-6
     np.testing.assert_array_equal(out["packed"], o.pack(out["codes"], bits))
     np.testing.assert_array_equal(out["g_idx"], ref["g_idx"])
 
