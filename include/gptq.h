@@ -188,9 +188,10 @@ gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits
  * itself allocates nothing (no cudaMalloc, no cudaFree, no allocating library call).
  *  - cols > GPTQ_STATIC_MAX_COLS returns GPTQ_ERR_WORKSPACE before anything runs;
  *    use gptq_prepare with a caller workspace for larger layers.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current and caches it; make that first
- *    call before any stream capture.
+ *  - The first call in a device's context looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current and caches it with the
+ *    context's id; make that first call before any stream capture.  After a
+ *    device reset (a new context) the next call looks the address up again.
  *  - Every call shares the one array, which keeps the previous call's contents (the
  *    call clears what must start at zero itself).  Calls whose work overlaps on the
  *    GPU — e.g. on two streams at once — race on the array; order them on one stream

@@ -24,7 +24,8 @@ using namespace gptq;
 
 static bool valid_dtype(int dt) { return dt == GPTQ_F32 || dt == GPTQ_F16 || dt == GPTQ_BF16; }
 
-static gptq_status check_cfg(const gptq_config* cfg) {
+namespace gptq {
+gptq_status check_cfg(const gptq_config* cfg) {
   if (!cfg) return GPTQ_ERR_INVALID_ARG;
   if (cfg->bits != 2 && cfg->bits != 3 && cfg->bits != 4 && cfg->bits != 8)
     return GPTQ_ERR_INVALID_ARG;
@@ -36,6 +37,7 @@ static gptq_status check_cfg(const gptq_config* cfg) {
   if (cfg->group_size < -1) return GPTQ_ERR_INVALID_ARG;
   return GPTQ_OK;
 }
+}  // namespace gptq
 
 static gptq_status check_group(const gptq_config* cfg) {
   const int g = cfg->group_size;

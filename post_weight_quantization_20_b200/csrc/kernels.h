@@ -4,6 +4,9 @@
 
 namespace gptq {
 
+// abi.cu: validation of a gptq_config shared by every entry point that takes one
+gptq_status check_cfg(const gptq_config* cfg);
+
 // hessian.cu
 gptq_status hessian_prescale(cudaStream_t st, float* H, int C, double alpha, bool overwrite);
 gptq_status hessian_syrk_simt(cudaStream_t st, float* H, const void* X, int dt, int64_t m, int C,

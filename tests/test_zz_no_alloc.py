@@ -5,7 +5,10 @@ the device memory, code with a fixed memory budget, a service that must not
 allocate after start-up) cannot hand the library a workspace; this entry point
 uses a scratch array compiled into the library instead.  The test calls it
 through the C ABI twice in a row, on two different layers, and checks each result
-against gptq_prepare with a caller workspace.  It lives in its own file, collected
+against gptq_prepare with a caller workspace; that a call after a warm-up one
+changes neither the device's free memory nor torch's reserved memory; and that a
+call with a caller-given order right after a descending-diagonal call (whose
+leftovers share the array) still checks and uses the given order.  It lives in its own file, collected
 last, and passes both alone in a fresh process and after the other tests.
 """
 import numpy as np
@@ -71,3 +74,46 @@ def test_static_scratch_refuses_layers_above_its_limit():
     with pytest.raises(G.GPTQError) as e:
         G.gptq_prepare_static(H, G.make_config(4, 128), U, perm)
     assert e.value.code == G.GPTQ_ERR_WORKSPACE
+
+
+def test_static_scratch_allocates_nothing():
+    H = _hessian(512, 3)
+    cfg = G.make_config(4, 128, act_order=True)
+    U = torch.empty(512, 512, device=DEV)
+    perm = torch.empty(512, dtype=torch.int32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    G.gptq_prepare_static(H, cfg, U, perm, st)          # warm-up: the one-time set-up
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    reserved0 = torch.cuda.memory_reserved()
+    G.gptq_prepare_static(H, cfg, U, perm, st)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_reserved() == reserved0
+    assert int(st.item()) == 0
+
+
+def test_static_scratch_given_order_after_descending_order():
+    C = 384
+    H = _hessian(C, 4)
+    _static(H, G.make_config(4, 128, act_order=True))     # leaves its counts in the array
+    given = torch.from_numpy(np.random.default_rng(5).permutation(C).astype(np.int32)).to(DEV)
+    cfg = G.make_config(4, 128, act_order=G.GPTQ_ORDER_GIVEN)
+    U = torch.empty(C, C, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    G.gptq_prepare_static(H, cfg, U, given.clone(), st)
+    ref_perm = given.clone()
+    Uw = torch.empty(C, C, device=DEV)
+    sw = torch.zeros(1, dtype=torch.int32, device=DEV)
+    G.gptq_prepare(H, cfg, Uw, ref_perm, G.alloc_workspace(G.GPTQ_OP_PREPARE, 0, C, cfg, DEV), sw)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0 and int(sw.item()) == 0
+    assert _rel(U, Uw) <= U_TOL
+    # a bad permutation is still caught after a call that left other counts behind
+    bad = given.clone()
+    bad[3] = bad[4]
+    st2 = torch.zeros(1, dtype=torch.int32, device=DEV)
+    G.gptq_prepare_static(H, cfg, U, bad, st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) & G.GPTQ_ERR_INVALID_ARG
