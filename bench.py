@@ -1,13 +1,20 @@
 """Benchmark of the GPTQ layer solver (Hessian + prepare + sweep + pack per layer).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload opt125m]
+                    [--workload opt175b]
+    python bench.py --op hessian|prepare|quantize|layer --rows R --cols C --tokens T
 
 One step quantizes every layer of the workload once: Hessian accumulation over
 all calibration tokens, damping / ordering / inverse Cholesky factor, the
-blocked column sweep, and bit packing.  Inputs are seeded synthetic tensors
-resident in HBM before timing; the calibration set (2.4 GB for the default
-workload) is larger than L2, so no flush is needed between steps.
+blocked column sweep, and bit packing.  The default workload is the largest that
+fits one GPU: the OPT-175B-shaped layers (12288 x 12288, 49152 x 12288 and
+12288 x 49152, 262144 calibration tokens each, 38.6 GB of fp16 activations).
+Inputs are seeded synthetic tensors resident in HBM before timing; every layer's
+calibration set is larger than L2, so no flush is needed between steps.
+
+``--op`` times one stage of one layer on device-drawn inputs (X ~ N(0, 1) fp16,
+W ~ N(0, 0.02^2) fp16) and prints one text line: a small fixed command to put
+under a profiler (the untimed repeats are the warm-up a profiler skips with -s).
 
 Multi-GPU: one process per GPU (torchrun).  The path has no exchange step, so
 every rank quantizes its own replica of the workload (weak scaling); the only
@@ -37,10 +44,9 @@ from post_weight_quantization_20_b200.workloads import WORKLOADS  # noqa: E402
 METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per Hessian launch from an ncu capture of the current
-# kernel (a small case scaled to the bench's launch by the token count), or None.
-# The capture summarised in profiles/hessian_tc_C3072_T65536.md (C = 3072, 65536
-# tokens: 734.9 MB + 135.5 MB) predates the kernel's abort-path drain, so the
-# figure stays None until the kernel is captured again.
+# kernel, as bytes per token at the captured column count (a small case, scaled
+# to the bench's launch by the token count), or None when the kernel has changed
+# since its last capture.
 HESSIAN_TRAFFIC = None
 
 
@@ -250,6 +256,18 @@ def run_ours(args, rank, world, local_rank):
         return t.pin_memory()
 
     stream = torch.cuda.current_stream(dev)
+    # The layers run one after another on one stream, so they share one set of
+    # Hessian, factor and workspace buffers sized for the largest layer; only
+    # each layer's W, X and outputs are its own.
+    Rmax = max(l.rows for l, _, _ in host)
+    Cmax = max(l.cols for l, _, _ in host)
+    shared = {
+        "H": torch.empty(Cmax * Cmax, device=dev), "U": torch.empty(Cmax * Cmax, device=dev),
+        "perm": torch.empty(Cmax, dtype=torch.int32, device=dev),
+        "wsp": G.alloc_workspace(G.GPTQ_OP_PREPARE, Rmax, Cmax, cfg, dev),
+        "wsq": torch.empty(max(G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, l.rows, l.cols, cfg)
+                               for l, _, _ in host), dtype=torch.uint8, device=dev),
+    }
     layers = []
     for l, W, X in host:
         R, C = l.rows, l.cols
@@ -257,10 +275,10 @@ def run_ours(args, rank, world, local_rank):
         b = {
             "R": R, "C": C,
             "W": to_dev(W, wl.wdtype), "X": to_dev(X, wl.xdtype),
-            "H": torch.empty(C, C, device=dev), "U": torch.empty(C, C, device=dev),
-            "perm": torch.empty(C, dtype=torch.int32, device=dev),
-            "wsp": G.alloc_workspace(G.GPTQ_OP_PREPARE, R, C, cfg, dev),
-            "wsq": G.alloc_workspace(G.GPTQ_OP_QUANTIZE, R, C, cfg, dev),
+            "H": shared["H"][:C * C].view(C, C), "U": shared["U"][:C * C].view(C, C),
+            "perm": shared["perm"][:C],
+            "wsp": shared["wsp"],
+            "wsq": shared["wsq"][:G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, R, C, cfg)],
             "codes": torch.empty(R, C, dtype=torch.uint8, device=dev),
             "scales": torch.empty(R, Gn, device=dev), "zeros": torch.empty(R, Gn, device=dev),
             "g_idx": torch.empty(C, dtype=torch.int32, device=dev),
@@ -357,7 +375,12 @@ def run_ours(args, rank, world, local_rank):
     hess_flop = sum(float(m) * C * (C + 1) for _, _, m, C in hess_ev)
     n_hess = len(hess_ev)
 
-    # end to end through the public API from pinned host buffers
+    # end to end through the public API from pinned host buffers; the device-resident
+    # inputs and buffers of the timed steps are released first (the host path
+    # allocates its own)
+    layers.clear()
+    shared.clear()
+    torch.cuda.empty_cache()
     pinned = [(l, to_pinned(W, wl.wdtype), to_pinned(X, wl.xdtype)) for l, W, X in host]
     h2d = sum(w.numel() * w.element_size() + x.numel() * x.element_size() for _, w, x in pinned)
 
@@ -378,13 +401,17 @@ def run_ours(args, rank, world, local_rank):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     e2e_steps = max(1, min(args.steps, 5))
-    d2h = 0
     for _ in range(e2e_steps):
         outs = e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     d2h = sum(o.nbytes for o in outs)
+    e2e_status = 0
+    for o_ in outs:
+        e2e_status |= int(o_.status.item())
+    if status_over_ranks(e2e_status, world, dev):
+        raise RuntimeError(f"device status {G.status_names(e2e_status)} in the end-to-end steps")
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, dev)
@@ -394,9 +421,10 @@ def run_ours(args, rank, world, local_rank):
     achieved = hess_flop / (hess_ms * 1e-3) / 1e12 if hess_ms > 0 else None
     peak = float(peaks["bf16_tflops"])
     traffic = None
-    if HESSIAN_TRAFFIC and any(C == 3072 for _, _, _, C in hess_ev):
-        toks = [m for _, _, m, C in hess_ev if C == 3072][0]
-        traffic = HESSIAN_TRAFFIC["bytes_per_token_C3072"] * toks
+    if HESSIAN_TRAFFIC:
+        toks = [m for _, _, m, C in hess_ev if C == HESSIAN_TRAFFIC["cols"]]
+        if toks:
+            traffic = HESSIAN_TRAFFIC["bytes_per_token"] * toks[0]
     out = {
         "metric": METRIC,
         "value": job_ms_per_layer(ms, args.steps, len(layers), world),
@@ -417,8 +445,8 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "traffic_scope": ("bytes per C=3072 launch (the largest Hessian of the "
-                                       "workload), ncu capture at 65536 tokens scaled by tokens")
+                     "traffic_scope": (f"bytes per C={HESSIAN_TRAFFIC['cols']} launch, from an "
+                                       "ncu capture of a smaller token count scaled by tokens")
                      if traffic is not None else
                      "null: the kernel changed after its last ncu capture",
                      "peak_source": f"{peaks['source']} bf16 dense burst"},
@@ -431,22 +459,21 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------------- oracle arm
-# Tokens of each layer's calibration input the oracle's Hessian is timed on; the
-# Hessian's work is linear in tokens, so its time is scaled to the full count.
-SAMPLE_TOKENS = 16384
-
-
-def oracle_layer(W, X, wl, q):
-    """The float64 oracle on one layer; returns (seconds in the Hessian, seconds in
-    damping, factorization, sweep and pack)."""
-    from oracle import gptq_ref as o
-    t0 = time.perf_counter()
-    H, n = o.hessian(S.to_f64(X, wl.xdtype))
-    t1 = time.perf_counter()
-    out = o.gptq_quantize(S.to_f64(W, wl.wdtype), H, q.bits, q.group_size, q.sym, q.act_order,
-                          q.damp, q.block_size)
-    o.pack(out["codes"], q.bits)
-    return t1 - t0, time.perf_counter() - t1
+# The float64 oracle cannot run a full-size layer in a bounded time (at 49152
+# columns its factorization alone is ~3e14 flop and its matrices 19 GB each), so
+# each step runs one sub-problem, drawn from the workload's largest layer, and
+# every layer's time is extrapolated from it by each phase's work formula:
+#   Hessian      SAMPLE_TOKENS tokens x SAMPLE_COLS columns; work N C^2, scaled by
+#                (N / m) (C / Cs)^2;
+#   prepare      damping, order and factor of that Cs x Cs Hessian; work C^3,
+#                scaled by (C / Cs)^3;
+#   sweep        SAMPLE_ROWS rows at Cs/2 and at Cs columns, fitted as a C + b C^2
+#                (per-column vector work and the lazy trailing update) and
+#                evaluated at C, scaled by R / r;
+#   pack         r rows x Cs columns, scaled by (R / r)(C / Cs).
+SAMPLE_TOKENS = 8192
+SAMPLE_COLS = 3072
+SAMPLE_ROWS = 768
 
 
 def blas_threads():
@@ -459,59 +486,161 @@ def blas_threads():
 
 
 def cpu_sample(wl):
-    """A bounded sample of the workload for the oracle: every layer, with its first
-    SAMPLE_TOKENS calibration tokens."""
+    """One sub-problem of the workload's largest layer: (layer, W sample r x Cs, X sample
+    m x Cs, m, Cs, r)."""
+    l = max(wl.layers, key=lambda x: x.rows * x.cols * x.cols)
     m = min(wl.tokens, SAMPLE_TOKENS)
-    layers = []
-    for l in wl.layers:
-        W = S.gen_weight(l.rows, l.cols, wl.wdtype, wl.wspec, seed=1234, tag=l.tag)
-        X = S.gen_activations(m, l.cols, wl.xdtype, wl.xspec, seed=1234, tag=l.tag)
-        layers.append((l, W, X))
-    return m, layers
+    cs = min(l.cols, SAMPLE_COLS)
+    r = min(l.rows, SAMPLE_ROWS)
+    W = S.gen_weight(r, l.cols, wl.wdtype, wl.wspec, seed=1234, tag=l.tag)[:, :cs]
+    X = S.gen_activations(m, l.cols, wl.xdtype, wl.xspec, seed=1234, tag=l.tag)[:, :cs]
+    return l, np.ascontiguousarray(W), np.ascontiguousarray(X), m, cs, r
 
 
-def cpu_step_ms_per_layer(wl, m, layers):
-    """One step of the oracle over the sample, in ms per layer of the full workload:
-    each Hessian time scaled by tokens / m, the rest as measured."""
-    q = wl.quant[0]
-    total = 0.0
-    for l, W, X in layers:
-        th, tr = oracle_layer(W, X, wl, q)
-        total += th * (wl.tokens / m) + tr
-    return total / len(layers) * 1e3
+def oracle_phases(W, X, wl, q):
+    """Seconds the oracle spends on the sample: Hessian, prepare, sweep at Cs/2 and at
+    Cs columns, pack."""
+    from oracle import gptq_ref as o
+    t0 = time.perf_counter()
+    H, n = o.hessian(S.to_f64(X, wl.xdtype))
+    t1 = time.perf_counter()
+    perm, Hp, U = o.prepare(H, q.damp, q.act_order)
+    t2 = time.perf_counter()
+    Wp = S.to_f64(W, wl.wdtype)[:, perm]
+    half = max(1, W.shape[1] // 2)
+    o.sweep(Wp[:, :half], U[:half, :half], q.bits, q.group_size, q.sym, q.block_size)
+    t3 = time.perf_counter()
+    res = o.sweep(Wp, U, q.bits, q.group_size, q.sym, q.block_size)
+    t4 = time.perf_counter()
+    o.pack(res["codes"], q.bits)
+    t5 = time.perf_counter()
+    return t1 - t0, t2 - t1, t3 - t2, t4 - t3, t5 - t4
 
 
-def cpu_sample_text(wl, m, layers):
-    names = ", ".join(f"{l.name} {l.rows}x{l.cols}" for l, _, _ in layers)
-    scale = "" if m == wl.tokens else (
-        f"; each Hessian on the first {m} of {wl.tokens} calibration tokens, its time "
-        f"scaled by {wl.tokens / m:g} (its work is linear in tokens)")
-    what = f"all {len(layers)} layers" if len(layers) > 1 else "the one layer"
-    return (f"per step {what} of the workload ({names}){scale}; damping, "
-            f"factorization, sweep and pack timed in full; float64 NumPy oracle on host cores")
+def sweep_model(t_half, t_full, c_half, c_full, C):
+    """Fit t(c) = a c + b c^2 through the two sweep samples (a, b >= 0) and evaluate it
+    at C."""
+    # solve [c1 c1^2; c2 c2^2] [a b]^T = [t1 t2]^T
+    det = c_half * c_full ** 2 - c_full * c_half ** 2
+    if det <= 0:
+        return t_full * C / c_full
+    a = (t_half * c_full ** 2 - t_full * c_half ** 2) / det
+    b = (c_half * t_full - c_full * t_half) / det
+    if a < 0 or b < 0:       # timing noise: keep the single-term fit that stays non-negative
+        a, b = (t_full / c_full, 0.0) if b < 0 else (0.0, t_full / c_full ** 2)
+    return a * C + b * C * C
+
+
+def layer_ms_from_sample(times, l, wl, m, cs, r):
+    """One full layer's oracle time (ms), extrapolated from the sample's phase times."""
+    th, tp, ts1, ts2, tk = times
+    C, R, N = l.cols, l.rows, wl.tokens
+    half = max(1, cs // 2)
+    total = (th * (N / m) * (C / cs) ** 2 + tp * (C / cs) ** 3 +
+             sweep_model(ts1, ts2, half, cs, C) * (R / r) + tk * (R / r) * (C / cs))
+    return total * 1e3
+
+
+def cpu_step_ms_per_layer(wl, sample):
+    """One oracle step: the sample timed once, every layer extrapolated from it; the
+    mean over the workload's layers (ms per layer)."""
+    _, W, X, m, cs, r = sample
+    times = oracle_phases(W, X, wl, wl.quant[0])
+    return sum(layer_ms_from_sample(times, l, wl, m, cs, r) for l in wl.layers) / len(wl.layers)
+
+
+def cpu_sample_text(wl, sample):
+    l, _, _, m, cs, r = sample
+    return (f"per step one sub-problem of the {l.rows}x{l.cols} layer ({m} tokens, {cs} cols, "
+            f"{r} rows of its inputs); every layer of the workload extrapolated from it by "
+            f"each phase's work: Hessian x (N/m)(C/Cs)^2, prepare x (C/Cs)^3, sweep fitted as "
+            f"a C + b C^2 from Cs/2 and Cs columns and x R/r, pack x (R/r)(C/Cs); float64 "
+            f"NumPy oracle on host cores")
 
 
 def run_cpu_baseline(wl):
-    m, layers = cpu_sample(wl)
-    v = cpu_step_ms_per_layer(wl, m, layers)
+    sample = cpu_sample(wl)
+    v = cpu_step_ms_per_layer(wl, sample)
     return {"value": v, "unit": "ms per layer", "cores": blas_threads(), "kind": "oracle",
-            "sample": "one step: " + cpu_sample_text(wl, m, layers)}
+            "sample": "one step: " + cpu_sample_text(wl, sample)}
 
 
 def run_reference(args):
     wl = WORKLOADS[args.workload]
-    m, layers = cpu_sample(wl)
+    sample = cpu_sample(wl)
     for _ in range(args.warmup):
-        cpu_step_ms_per_layer(wl, m, layers)
-    v = sum(cpu_step_ms_per_layer(wl, m, layers) for _ in range(args.steps)) / max(args.steps, 1)
+        cpu_step_ms_per_layer(wl, sample)
+    v = sum(cpu_step_ms_per_layer(wl, sample) for _ in range(args.steps)) / max(args.steps, 1)
     cores = blas_threads()
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "ms", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * len(layers),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": v * len(wl.layers),
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded)", "config": workload_config(wl, 1),
             "cpu_baseline": {"value": v, "unit": "ms per layer", "cores": cores, "kind": "oracle",
-                             "sample": cpu_sample_text(wl, m, layers)},
+                             "sample": cpu_sample_text(wl, sample)},
             "e2e": {"value": v, "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- one stage
+def run_op(args):
+    """Time one stage of one layer on device-drawn inputs; one text line."""
+    import torch
+    from post_weight_quantization_20_b200 import gptq as G
+    dev = torch.device("cuda", torch.cuda.current_device())
+    G.load_library()
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    R, C, T = args.rows, args.cols, args.tokens
+    X = torch.randn(T, C, device=dev, generator=gen).half()
+    W = (0.02 * torch.randn(R, C, device=dev, generator=gen)).half()
+    cfg = G.make_config(args.bits, args.group, act_order=args.act_order)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    H = torch.empty(C, C, device=dev)
+    U = torch.empty(C, C, device=dev)
+    perm = torch.empty(C, dtype=torch.int32, device=dev)
+    wsp = G.alloc_workspace(G.GPTQ_OP_PREPARE, R, C, cfg, dev)
+    G.gptq_hessian_accumulate(H, 0, X, status)
+    if args.op == "hessian":
+        def run():
+            G.gptq_hessian_accumulate(H, 0, X, status)
+        work = f"{float(T) * C * (C + 1) / 1e12:.4f} TFLOP per call"
+    elif args.op == "prepare":
+        def run():
+            G.gptq_prepare(H, cfg, U, perm, wsp, status)
+        work = f"{2.0 * C ** 3 / 3e12:.4f} TFLOP per call (2/3 C^3)"
+    elif args.op == "quantize":
+        G.gptq_prepare(H, cfg, U, perm, wsp, status)
+        Gn = G.n_groups(C, cfg.group_size)
+        codes = torch.empty(R, C, dtype=torch.uint8, device=dev)
+        scales = torch.empty(R, Gn, device=dev)
+        zeros = torch.empty(R, Gn, device=dev)
+        g_idx = torch.empty(C, dtype=torch.int32, device=dev)
+        losses = torch.empty(C, device=dev)
+        packed = torch.empty(R, G.packed_words(C, cfg.bits), dtype=torch.int32, device=dev)
+        wsq = G.alloc_workspace(G.GPTQ_OP_QUANTIZE, R, C, cfg, dev)
+
+        def run():
+            G.gptq_quantize_layer(W, U, perm, cfg, codes, scales, zeros, g_idx, losses, wsq, status)
+            G.gptq_pack(codes, cfg.bits, packed)
+        work = f"sweep + lazy updates + pack, {float(R) * C * C / 1e12:.4f} TFLOP of update per call"
+    else:
+        def run():
+            G.quantize_layer(W, X, cfg, check=False)
+        work = "Hessian + prepare + sweep + pack, with their allocations"
+    for _ in range(args.repeat):
+        run()
+    torch.cuda.synchronize(dev)
+    G.check_status(status, args.op)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.repeat):
+        run()
+    e1.record()
+    torch.cuda.synchronize(dev)
+    G.check_status(status, args.op)
+    ms = e0.elapsed_time(e1) / args.repeat
+    print(f"op={args.op} rows={R} cols={C} tokens={T}: {ms:.3f} ms per call ({work})", flush=True)
 
 
 def main():
@@ -520,9 +649,21 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="opt125m", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="opt175b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="step", choices=["step", "hessian", "prepare", "quantize",
+                                                     "layer"])
+    ap.add_argument("--rows", type=int, default=768)
+    ap.add_argument("--cols", type=int, default=3072)
+    ap.add_argument("--tokens", type=int, default=16384)
+    ap.add_argument("--repeat", type=int, default=3)
+    ap.add_argument("--bits", type=int, default=4)
+    ap.add_argument("--group", type=int, default=128)
+    ap.add_argument("--act-order", action="store_true")
     args = ap.parse_args()
+    if args.op != "step":
+        run_op(args)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -84,13 +84,23 @@ def hessian_accumulate(H: np.ndarray, n: int, X: np.ndarray):
 
 
 def hessian(X: np.ndarray, chunk: int | None = None):
-    """H = 2/n X^T X over all tokens of X, accumulated chunk by chunk."""
+    """H = 2/n X^T X over all tokens of X, accumulated chunk by chunk with the same
+    running-mean update as hessian_accumulate (each entry rounded the same way; the
+    update is done in place on H so that a wide layer needs no C x C temporaries
+    beyond the chunk's X^T X)."""
     cols = X.shape[1]
     H = np.zeros((cols, cols))
     n = 0
     step = chunk or max(1, X.shape[0])
     for t in range(0, X.shape[0], step):
-        H, n = hessian_accumulate(H, n, X[t:t + step])
+        Xd = np.asarray(X[t:t + step], dtype=np.float64)
+        m = int(Xd.shape[0])
+        G = Xd.T @ Xd
+        G *= 2.0 / (n + m)
+        H *= n / (n + m)
+        H += G
+        del G
+        n += m
     return H, n
 
 

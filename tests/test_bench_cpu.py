@@ -1,5 +1,5 @@
 """bench.py's host-side parts that need no GPU: the reference arm's JSON line, the
-scaling of the oracle's sampled Hessian time, and the L2 statement."""
+scaling of the oracle's sampled phase times to the full layer, and the L2 statement."""
 import json
 import subprocess
 import sys
@@ -31,18 +31,31 @@ def test_reference_arm_prints_one_contract_line():
                           "d2h_bytes_per_step": 0}
 
 
-def test_sampled_hessian_time_is_scaled_to_the_full_token_count(monkeypatch):
-    wl = WORKLOADS["opt125m"]
-    m = bench.SAMPLE_TOKENS
-    times = {768: (0.5, 1.0), 3072: (2.0, 3.0)}     # (Hessian s, rest s) by cols
-    monkeypatch.setattr(bench, "oracle_layer", lambda W, X, wl_, q: times[X.shape[1]])
-    layers = [(l, None, SimpleNamespace(shape=(m, l.cols))) for l in wl.layers]
-    got = bench.cpu_step_ms_per_layer(wl, m, layers)
-    scale = wl.tokens / m
-    want = sum(times[l.cols][0] * scale + times[l.cols][1] for l in wl.layers) / 3 * 1e3
-    assert got == pytest.approx(want, rel=1e-12)
-    assert scale == 16
-    assert "scaled by 16" in bench.cpu_sample_text(wl, m, layers)
+def test_sampled_phase_times_are_scaled_to_the_full_layer(monkeypatch):
+    wl = WORKLOADS["opt175b"]
+    l = wl.layers[2]                                   # 12288 x 49152
+    m, cs, r = bench.SAMPLE_TOKENS, bench.SAMPLE_COLS, bench.SAMPLE_ROWS
+    # sweep times exactly a c + b c^2 with a = 1e-5, b = 1e-9: the fit must recover it
+    a, b = 1e-5, 1e-9
+    times = (0.5, 2.0, a * cs / 2 + b * (cs / 2) ** 2, a * cs + b * cs ** 2, 0.01)
+    got = bench.layer_ms_from_sample(times, l, wl, m, cs, r)
+    C, R, N = l.cols, l.rows, wl.tokens
+    want = (0.5 * (N / m) * (C / cs) ** 2 + 2.0 * (C / cs) ** 3 +
+            (a * C + b * C * C) * (R / r) + 0.01 * (R / r) * (C / cs)) * 1e3
+    assert got == pytest.approx(want, rel=1e-9)
+    text = bench.cpu_sample_text(wl, (l, None, None, m, cs, r))
+    assert "extrapolated" in text and f"{m} tokens, {cs} cols, {r} rows" in text
+    # the step: one timed sample, every layer extrapolated from it, the mean per layer
+    monkeypatch.setattr(bench, "oracle_phases", lambda W, X, wl_, q: times)
+    step = bench.cpu_step_ms_per_layer(wl, (l, None, None, m, cs, r))
+    assert step == pytest.approx(sum(bench.layer_ms_from_sample(times, x, wl, m, cs, r)
+                                     for x in wl.layers) / 3, rel=1e-12)
+
+
+def test_sweep_fit_stays_non_negative():
+    # noise that would give a negative quadratic term falls back to a linear fit
+    assert bench.sweep_model(0.6, 1.0, 100, 200, 400) == pytest.approx(2.0)
+    assert bench.sweep_model(0.25, 1.0, 100, 200, 400) == pytest.approx(4.0)
 
 
 def test_l2_statement_follows_the_input_size():

@@ -104,7 +104,7 @@ def _prep_gpu(H32, cfg, perm=None):
     return U.cpu().numpy().astype(np.float64), p.cpu().numpy(), int(st.item())
 
 
-@pytest.mark.parametrize("cols", [1, 63, 128, 200, 520])
+@pytest.mark.parametrize("cols", [1, 63, 128, 200, 520, 1600, 2200])
 @pytest.mark.parametrize("act", [False, True])
 def test_prepare_matches_oracle(cols, act):
     X = S.gen_activations(4 * cols + 64, cols, S.F32, S.ActSpec(dist="t4", mix_rank=3), seed=cols)
@@ -116,6 +116,7 @@ def test_prepare_matches_oracle(cols, act):
     perm_o, Hp, Uo = o.prepare(H32.astype(np.float64), 0.01, act)
     np.testing.assert_array_equal(perm, perm_o)
     assert np.all(np.tril(U, -1) == 0) and np.all(np.diag(U) > 0)
+    print(f"prepare cols={cols} act={act}: U rel Frobenius {rel_fro(U, Uo):.2e}")
     assert rel_fro(U, Uo) <= 1e-3
 
 
