@@ -263,7 +263,6 @@ def run_ours(args, rank, world, local_rank):
     Cmax = max(l.cols for l, _, _ in host)
     shared = {
         "H": torch.empty(Cmax * Cmax, device=dev), "U": torch.empty(Cmax * Cmax, device=dev),
-        "perm": torch.empty(Cmax, dtype=torch.int32, device=dev),
         "wsp": G.alloc_workspace(G.GPTQ_OP_PREPARE, Rmax, Cmax, cfg, dev),
         "wsq": torch.empty(max(G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, l.rows, l.cols, cfg)
                                for l, _, _ in host), dtype=torch.uint8, device=dev),
@@ -276,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
             "R": R, "C": C,
             "W": to_dev(W, wl.wdtype), "X": to_dev(X, wl.xdtype),
             "H": shared["H"][:C * C].view(C, C), "U": shared["U"][:C * C].view(C, C),
-            "perm": shared["perm"][:C],
+            "perm": torch.empty(C, dtype=torch.int32, device=dev),
             "wsp": shared["wsp"],
             "wsq": shared["wsq"][:G.gptq_workspace_size(G.GPTQ_OP_QUANTIZE, R, C, cfg)],
             "codes": torch.empty(R, C, dtype=torch.uint8, device=dev),
@@ -375,9 +374,13 @@ def run_ours(args, rank, world, local_rank):
     hess_flop = sum(float(m) * C * (C + 1) for _, _, m, C in hess_ev)
     n_hess = len(hess_ev)
 
+    stored = stored_form_product(G, layers, cfg, dev, stream, args)
+    group = shared_input_group(G, layers[0], wl, cfg, dev, stream, args, to_dev)
+
     # end to end through the public API from pinned host buffers; the device-resident
     # inputs and buffers of the timed steps are released first (the host path
     # allocates its own)
+    n_layers_rank = len(layers)
     layers.clear()
     shared.clear()
     torch.cuda.empty_cache()
@@ -427,7 +430,7 @@ def run_ours(args, rank, world, local_rank):
             traffic = HESSIAN_TRAFFIC["bytes_per_token"] * toks[0]
     out = {
         "metric": METRIC,
-        "value": job_ms_per_layer(ms, args.steps, len(layers), world),
+        "value": job_ms_per_layer(ms, args.steps, n_layers_rank, world),
         "unit": "ms",
         "n_gpus": world,
         "steps": args.steps,
@@ -450,12 +453,106 @@ def run_ours(args, rank, world, local_rank):
                      if traffic is not None else
                      "null: the kernel changed after its last ncu capture",
                      "peak_source": f"{peaks['source']} bf16 dense burst"},
-        "e2e": {"value": e2e_ms / len(layers), "unit": "ms", "h2d_bytes_per_step": int(h2d),
+        "e2e": {"value": e2e_ms / n_layers_rank, "unit": "ms", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
+        "stored_form": stored,
+        "shared_input_group": group,
         "gpu_launches": int(launches),
         "clocks": cl,
     }
     return out
+
+
+# ----------------------------------------------------------------------------- stored form
+def stored_form_product(G, layers, cfg, dev, stream, args):
+    """The inference side of the quantized layers: Y = X Q^T for one decode token from
+    each layer's packed codes (repacked to sweep order once), timed over all layers
+    with CUDA events.  HBM-bound: per layer it reads R C b/8 bytes of codes and R G 8
+    of grids (plus the token and the output)."""
+    import torch
+    peaks = load_peaks()
+    items, nbytes = [], 0
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1)
+    for b in layers:
+        R, C = b["R"], b["C"]
+        qp = torch.empty(R, G.sweep_words(C, cfg.bits), dtype=torch.int32, device=dev)
+        G.gptq_repack_sweep_order(b["packed"], cfg.bits, b["perm"], qp, stream)
+        x = torch.randn(1, C, device=dev, generator=gen).half()
+        y = torch.empty(1, R, device=dev)
+        items.append((qp, b["scales"], b["zeros"], b["perm"], x, y))
+        nbytes += R * C * cfg.bits // 8 + b["scales"].numel() * 8 + C * 2 + R * 4
+    reps = max(3, min(args.steps, 20))
+
+    def run():
+        for qp, sc, ze, pm, x, y in items:
+            G.gptq_dequant_matmul(x, qp, sc, ze, cfg.bits, cfg.group_size, pm, y, stream=stream)
+    for _ in range(3):
+        run()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(reps):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1) / reps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"op": f"Y = x Q^T, one fp16 token, from the packed {cfg.bits}-bit codes of every "
+                  f"layer (sweep-order repack, fp32 sums)",
+            "ms_per_step": ms, "bytes_per_step": int(nbytes), "achieved_gbs": gbs,
+            "peak_gbs": float(peaks["hbm_gbs"]), "frac": gbs / float(peaks["hbm_gbs"]),
+            "peak_source": f"{peaks['source']} HBM copy"}
+
+
+# ----------------------------------------------------------------------------- shared input
+def shared_input_group(G, b, wl, cfg, dev, stream, args, to_dev):
+    """Layers that read the same input (the q, k and v projections of one attention
+    block): one Hessian and one factorization, then one sweep per weight, against the
+    same three layers quantized one by one.  The first layer of the workload and two
+    more weights of its shape, drawn from the same distribution."""
+    import torch
+    R, C = b["R"], b["C"]
+    l = wl.layers[0]
+    Ws = [b["W"]] + [to_dev(S.gen_weight(R, C, wl.wdtype, wl.wspec, seed=1234, tag=l.tag + 500 + k),
+                            wl.wdtype) for k in range(2)]
+
+    def sweep(W):
+        G.gptq_quantize_layer(W, b["U"], b["perm"], cfg, b["codes"], b["scales"], b["zeros"],
+                              b["g_idx"], b["losses"], b["wsq"], b["status"], stream)
+        G.gptq_pack(b["codes"], cfg.bits, b["packed"], stream)
+
+    def factor():
+        G.gptq_hessian_accumulate(b["H"], 0, b["X"], b["status"], stream)
+        G.gptq_prepare(b["H"], cfg, b["U"], b["perm"], b["wsp"], b["status"], stream)
+
+    def shared():
+        factor()
+        for W in Ws:
+            sweep(W)
+
+    def separate():
+        for W in Ws:
+            factor()
+            sweep(W)
+
+    reps = max(1, min(args.steps, 3))
+    out = {}
+    for name, fn in (("shared", shared), ("separate", separate)):
+        fn()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            fn()
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        out[name] = t0.elapsed_time(t1) / reps
+    if int(b["status"].item()):
+        raise RuntimeError(f"device status {G.status_names(int(b['status'].item()))} "
+                           "in the shared-input group")
+    return {"layers": f"3 x {R}x{C} reading one {wl.tokens}-token input",
+            "ms_per_layer_shared": out["shared"] / 3, "ms_per_layer_separate": out["separate"] / 3}
 
 
 # ----------------------------------------------------------------------------- oracle arm

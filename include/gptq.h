@@ -202,6 +202,43 @@ gptq_status gptq_pack(const uint8_t* codes, int64_t rows, int64_t cols, int bits
 gptq_status gptq_prepare_static(const float* H, int64_t cols, const gptq_config* cfg, float* U,
                                 int32_t* perm, int32_t* dev_status, void* stream);
 
+/*
+ * gptq_repack_sweep_order — the packed codes of gptq_pack (original column order)
+ * rewritten in sweep order for gptq_dequant_matmul: column j of an output row holds
+ * original column perm[j] (perm from gptq_prepare; NULL = identity).  Under
+ * act-order a group's columns are scattered over the original order (the gather
+ * desc_act costs at inference, GPTQ量化算法深度解析 §3.3); in sweep order every group
+ * is one contiguous run and the gather moves to the small activation block.
+ *  packed  rows x ceil(cols*bits/32) uint32 (gptq_pack layout)
+ *  out     rows x (cols/32)*bits uint32, same bitstream layout, sweep order
+ *  cols % 32 == 0, bits in {2,3,4,8}.  Errors: INVALID_ARG.
+ */
+gptq_status gptq_repack_sweep_order(const uint32_t* packed, int64_t rows, int64_t cols,
+                                    int bits, const int32_t* perm, uint32_t* out,
+                                    void* stream);
+/*
+ * gptq_dequant_matmul — Y = X Q^T from the stored form, decode-sized token counts
+ * (gptq-for-llama article, "工程细节": products straight from packed 4-bit codes):
+ *     Q[r][c] = scales[r][g(c)] (code[r][c] - zeros[r][g(c)])
+ *  X       m_tokens x cols, row stride ldx, xdtype, m_tokens >= 1 (decode-sized
+ *          counts run in one pass; larger ones in blocks of 8 tokens, each
+ *          reading the weights again)
+ *  qp      sweep-order codes from gptq_repack_sweep_order, 16-byte aligned
+ *  scales, zeros  rows x G fp32 from gptq_quantize_layer (groups in sweep order)
+ *  group_size 0 (per row), 32, 64 or 128; perm: sweep order (NULL = natural)
+ *  Y       m_tokens x rows fp32
+ *  half_sums  nonzero: for 4-bit codes, fp16 X and m_tokens <= 2, each 8-code word
+ *          is summed in half precision (half2 FMA; relative rounding 2^-11 per
+ *          step) before the fp32 grid step -- about half the instructions per code;
+ *          otherwise (or 0) every sum is fp32.
+ *  Errors: INVALID_ARG, UNSUPPORTED (other group sizes).
+ */
+gptq_status gptq_dequant_matmul(const void* X, int xdtype, int64_t m_tokens, int64_t cols,
+                                int64_t ldx, const uint32_t* qp, const float* scales,
+                                const float* zeros, int bits, int group_size,
+                                const int32_t* perm, float* Y, int64_t rows, int half_sums,
+                                void* stream);
+
 /* Self-test of the failure detection (the pages have no counterpart).  Launches a
  * kernel whose bounded device wait is made to run out, so that a caller or a test
  * can check that the wait gives up, OR-s GPTQ_ERR_TIMEOUT into *dev_status and
@@ -217,6 +254,16 @@ gptq_status gptq_prepare_static(const float* H, int64_t cols, const gptq_config*
 #define GPTQ_SELFTEST_MBARRIER 0
 #define GPTQ_SELFTEST_GRID_BARRIER 1
 gptq_status gptq_selftest_timeout(int which, int32_t* dev_status, void* stream);
+
+/* Diagnostic (the pages have no counterpart): the number of polls after which a
+ * wait in the tensor-core pipelines (the Hessian and the 3xTF32 products) gives up,
+ * for kernels launched after this call; 0 restores the default (about a second).
+ * With a small value the waits run out during normal work, so that a test can
+ * check that such a kernel stops its producer and MMA issuer, waits for the copies
+ * and MMAs it has in flight (those waits keep the default limit), frees its TMEM,
+ * OR-s GPTQ_ERR_TIMEOUT into the status word and leaves the context usable.
+ * Process-wide; returns the previous limit. */
+uint32_t gptq_debug_set_wait_limit(uint32_t polls);
 
 /* Human-readable name of a status code (static string). */
 const char* gptq_status_string(int status);

@@ -6,11 +6,17 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 #include <cstdio>
 
 namespace gptq {
 static std::atomic<uint64_t> g_launches{0};
+static std::atomic<uint32_t> g_wait_limit{0};   // 0: tc::WAIT_LIMIT
+uint32_t pipeline_wait_limit() {
+  const uint32_t v = g_wait_limit.load(std::memory_order_relaxed);
+  return v ? v : tc::WAIT_LIMIT;
+}
 static thread_local char g_last_error[256] = "";
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 void note_error(cudaError_t e, const char* where) {
@@ -141,6 +147,43 @@ gptq_status gptq_selftest_timeout(int which, int32_t* dev_status, void* stream) 
   if (which == GPTQ_SELFTEST_GRID_BARRIER)
     return selftest_grid_barrier(as_stream(stream), dev_status);
   return GPTQ_ERR_INVALID_ARG;
+}
+
+gptq_status gptq_repack_sweep_order(const uint32_t* packed, int64_t rows, int64_t cols, int bits,
+                                    const int32_t* perm, uint32_t* out, void* stream) {
+  CallRange range_("gptq_repack_sweep_order");
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (rows < 0 || rows > INT_MAX || cols <= 0 || cols > INT_MAX / 2 || cols % 32 != 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (rows > 0 && (!packed || !out)) return GPTQ_ERR_INVALID_ARG;
+  return repack_sweep_run(as_stream(stream), packed, int(rows), int(cols), bits, perm, out);
+}
+
+gptq_status gptq_dequant_matmul(const void* X, int xdtype, int64_t m_tokens, int64_t cols,
+                                int64_t ldx, const uint32_t* qp, const float* scales,
+                                const float* zeros, int bits, int group_size,
+                                const int32_t* perm, float* Y, int64_t rows, int half_sums,
+                                void* stream) {
+  CallRange range_("gptq_dequant_matmul");
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8) return GPTQ_ERR_INVALID_ARG;
+  if (rows < 0 || rows > INT_MAX || cols <= 0 || cols > INT_MAX / 2 || cols % 32 != 0)
+    return GPTQ_ERR_INVALID_ARG;
+  if (m_tokens < 1 || m_tokens > INT_MAX || !valid_dtype(xdtype) || ldx < cols)
+    return GPTQ_ERR_INVALID_ARG;
+  if (group_size != 0 && group_size != -1 && group_size != 32 && group_size != 64 &&
+      group_size != 128)
+    return GPTQ_ERR_UNSUPPORTED;
+  if (!X || !Y) return GPTQ_ERR_INVALID_ARG;
+  if (rows > 0 && (!qp || !scales || !zeros)) return GPTQ_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(qp) & 15) != 0) return GPTQ_ERR_INVALID_ARG;
+  return dequant_matmul_run(as_stream(stream), X, xdtype, int(m_tokens), int(cols), ldx, qp,
+                            scales, zeros, bits, group_size > 0 ? group_size : 0, perm, Y,
+                            int(rows), half_sums != 0);
+}
+
+uint32_t gptq_debug_set_wait_limit(uint32_t polls) {
+  const uint32_t old = g_wait_limit.exchange(polls, std::memory_order_relaxed);
+  return old ? old : tc::WAIT_LIMIT;
 }
 
 uint64_t gptq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -46,19 +46,43 @@ constexpr uint32_t TMEM_COLS = 2 * BN;
 
 struct Sched {
   int C, T, S, kt, ntj, vec;
+  uint32_t wait_limit;   // polls of an mbarrier wait before it gives up
 };
 
-// t-th upper tile: j-tile jt holds i-tiles a = 0 .. min(nti, 2 jt + 2) - 1.
+// Upper tiles: tile (it, jt) exists iff it < min(nti, 2 jt + 2), i.e. jt >= it / 2.
+// They are ordered in groups of GJ j-tiles (GJ * 256 columns); inside a group by
+// i-tile, then j-tile.  The tiles in flight together (one per SM) then cover about
+// 18 i-tiles x GJ j-tiles, 4.4k columns of X at 49152 columns instead of 19k for a
+// j-band order, so each token's columns come from HBM about four times less often.
+constexpr int GJ = 8;
+
+// number of tiles of group g (j-tiles jb0 .. jb1 - 1)
+__device__ __forceinline__ int group_tiles(int nti, int ntj, int g) {
+  const int jb0 = g * GJ, jb1 = min(jb0 + GJ, ntj);
+  const int imax = min(nti, 2 * jb1);
+  int n = 0;
+  for (int it = 0; it < imax; ++it) n += jb1 - max(jb0, it / 2);
+  return n;
+}
+
 __device__ __forceinline__ void tile_coords(const Sched& s, int t, int& i0, int& j0) {
   const int nti = (s.C + BM - 1) / BM;
-  int jt = 0;
-  for (; jt < s.ntj; ++jt) {
-    const int cnt = min(nti, 2 * jt + 2);
-    if (t < cnt) break;
-    t -= cnt;
+  const int ng = (s.ntj + GJ - 1) / GJ;
+  int g = 0;
+  for (; g < ng - 1; ++g) {
+    const int n = group_tiles(nti, s.ntj, g);
+    if (t < n) break;
+    t -= n;
   }
-  i0 = t * BM;
-  j0 = jt * BN;
+  const int jb0 = g * GJ, jb1 = min(jb0 + GJ, s.ntj);
+  int it = 0;
+  for (;; ++it) {
+    const int n = jb1 - max(jb0, it / 2);
+    if (t < n) break;
+    t -= n;
+  }
+  i0 = it * BM;
+  j0 = (max(jb0, it / 2) + t) * BN;
 }
 
 __device__ __forceinline__ void item_range(const Sched& s, int w, int& t, int& k0, int& k1) {
@@ -118,7 +142,7 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
         item_range(s, w, t, k0, k1);
         tile_coords(s, t, i0, j0);
         for (int k = k0; k < k1; ++k) {
-          if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(empty + stage, phase ^ 1u, abort_flag, s.wait_limit)) { ok = false; break; }
           uint8_t* a = smem + stage * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
           tc::mbar_expect_tx(full + stage, STAGE_BYTES);
@@ -144,11 +168,11 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
         item_range(s, w, t, k0, k1);
         for (int ks = k0; ks < k1 && ok; ks += SEG) {
           const int ke = min(ks + SEG, k1);
-          if (!tc::mbar_wait(acc_empty + acc, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+          if (!tc::mbar_wait(acc_empty + acc, acc_phase ^ 1u, abort_flag, s.wait_limit)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t d = tmem_base + uint32_t(acc * BN);
           for (int k = ks; k < ke; ++k) {
-            if (!tc::mbar_wait(full + stage, phase, abort_flag)) { ok = false; break; }
+            if (!tc::mbar_wait(full + stage, phase, abort_flag, s.wait_limit)) { ok = false; break; }
             tc::fence_after_sync();
             const uint8_t* a = smem + stage * STAGE_BYTES;
             const uint8_t* b = a + A_BYTES;
@@ -184,7 +208,7 @@ k_hess_syrk_tc(const __grid_constant__ CUtensorMap xmap, float* H, Sched s, floa
 #pragma unroll
       for (int q = 0; q < 128; ++q) r[q] = 0.f;
       for (int ks = k0; ks < k1; ks += SEG) {
-        if (!tc::mbar_wait(acc_full + acc, acc_phase, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(acc_full + acc, acc_phase, abort_flag, s.wait_limit)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -321,6 +345,7 @@ gptq_status hessian_syrk_tc(cudaStream_t st, float* H, const void* X, int dt, in
   s.kt = int((m + BK - 1) / BK);
   s.S = choose_splits(s.T, P, s.kt);
   s.vec = ((C & 3) == 0 && (reinterpret_cast<uintptr_t>(H) & 15) == 0) ? 1 : 0;
+  s.wait_limit = pipeline_wait_limit();
   const int items = s.S * s.T;
   const int grid = std::min(P, items);
 

@@ -23,12 +23,22 @@ constexpr int NB = 64;  // diagonal block of the factorization
 
 constexpr int MAX_FACTOR_GRID = 1024;   // CTAs of the persistent factorization (at most)
 
+// Above OUTER_MIN_COLS columns the factorization is blocked twice: the persistent
+// kernel runs OUTER_BLOCKS 64-column steps at a time inside an outer panel, and two
+// tensor-core products with K = 64 * OUTER_BLOCKS update the rest.
+constexpr int OUTER_BLOCKS = 8;
+constexpr int OUTER_K = OUTER_BLOCKS * 64;
+constexpr int OUTER_MIN_COLS = 3584;   // measured: at 3072 columns one launch is faster
+
 struct PrepLayout {
   int Cp, nblk;
   float *A, *Bx, *T, *diag, *lam;
   int32_t* cnt;
   int32_t* smid;   // [MAX_FACTOR_GRID]: the SM each CTA of the factorization runs on
+  float *Lh, *Ll, *Mh, *Ml;   // outer path: TF32 splits, Cp x OUTER_K each (else null)
 };
+
+static bool outer_path(int64_t Cp) { return Cp > OUTER_MIN_COLS; }
 
 static PrepLayout prep_layout(void* ws, int64_t C) {
   PrepLayout L{};
@@ -43,6 +53,13 @@ static PrepLayout prep_layout(void* ws, int64_t C) {
   L.lam = reinterpret_cast<float*>(p);          p += 256;
   L.cnt = reinterpret_cast<int32_t*>(p);        p += align256(size_t(C) * 4);
   L.smid = reinterpret_cast<int32_t*>(p);       p += align256(size_t(MAX_FACTOR_GRID) * 4);
+  if (outer_path(L.Cp)) {
+    const size_t sz = align256(size_t(L.Cp) * OUTER_K * 4);
+    L.Lh = reinterpret_cast<float*>(p);         p += sz;
+    L.Ll = reinterpret_cast<float*>(p);         p += sz;
+    L.Mh = reinterpret_cast<float*>(p);         p += sz;
+    L.Ml = reinterpret_cast<float*>(p);         p += sz;
+  }
   return L;
 }
 
@@ -50,7 +67,8 @@ size_t prepare_ws_bytes(int64_t C) {
   const int64_t nblk = (C + NB - 1) / NB, Cp = nblk * NB;
   const size_t cp2 = size_t(Cp) * Cp * sizeof(float);
   return 2 * align256(cp2) + align256(size_t(nblk) * NB * NB * 4) + align256(size_t(C) * 4) +
-         256 + align256(size_t(C) * 4) + align256(size_t(MAX_FACTOR_GRID) * 4);
+         256 + align256(size_t(C) * 4) + align256(size_t(MAX_FACTOR_GRID) * 4) +
+         (outer_path(Cp) ? 4 * align256(size_t(Cp) * OUTER_K * 4) : 0);
 }
 
 // lambda = damp * mean(diag H); flags a non-finite diagonal.
@@ -376,6 +394,8 @@ struct FactorArgs {
   int* abort_flag;     // set when a barrier gave up
   int32_t* status;
   int32_t* smid;       // [gridDim.x]
+  int kb, ke;          // the 64-column steps this launch runs, [kb, ke)
+  int lim;             // outer limit in blocks: SYRK columns and M^-1 rows stay below it
 };
 
 // Spins of a grid-barrier wait before it gives up (each a ~64 ns sleep and an
@@ -572,7 +592,8 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
     asm volatile("mov.u32 %0, %%smid;" : "=r"(id));
     a.smid[blockIdx.x] = int32_t(id);
   }
-  if (blockIdx.x == 0) diag_factor(a.A, lda, 0, a.T, a.status, sm);
+  if (blockIdx.x == 0)
+    diag_factor(a.A, lda, a.kb * NB, a.T + size_t(a.kb) * NB * NB, a.status, sm);
   if (!grid_barrier(a, epoch)) return;
   // CTA 0 carries the serial chain (the next diagonal block's update and factor).
   // A CTA that shares its SM would take half of its issue slots, so that CTA, if
@@ -590,7 +611,7 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
   const int nw = int(gridDim.x) - (idle >= 0 ? 1 : 0);                 // working CTAs
   const int rank = int(blockIdx.x) - (idle >= 0 && int(blockIdx.x) > idle ? 1 : 0);
   const bool works = int(blockIdx.x) != idle;
-  for (int k = 0; k < a.nblk; ++k) {
+  for (int k = a.kb; k < a.ke; ++k) {
     const int k0 = k * NB;
     const float* Tk = a.T + size_t(k) * NB * NB;
     const int rest = a.lda - k0 - NB;
@@ -617,18 +638,27 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
     };
     if (works) run_tiles64(rank, nw, nr + k + 1, phase_a, sm);
     if (!grid_barrier(a, epoch)) return;
-    if (rest == 0) break;
-    // phase B: A[k0+64:, k0+64:] -= P P^T (lower tiles) and
-    // Bx[k0+64:, 0:k0+64] -= P X_k
-    const int n_syrk = nr * (nr + 1) / 2;
-    const int n_total = n_syrk + nr * (k + 1);
+    if (rest == 0 || k + 1 >= a.lim) break;
+    // phase B: A[k0+64:, k0+64:lim] -= P P^T (lower tiles of the columns below the
+    // outer limit, all rows) and Bx[k0+64:lim, 0:k0+64] -= P X_k
+    const int ncol = a.lim - k - 1;                        // SYRK tile columns
+    const int n_syrk = ncol * nr - ncol * (ncol - 1) / 2;  // trapezoid: rows tn .. nr-1
+    const int nrb = ncol;                                  // M^-1 tile rows
+    const int n_total = n_syrk + nrb * (k + 1);
     float* trail = a.A + int64_t(k0 + NB) * lda + k0 + NB;
     float* bxb = a.Bx + int64_t(k0 + NB) * lda;
     const auto phase_b = [&](int t) {
       Tile64 T;
       int tm, tn;
       if (t < n_syrk) {
-        lower_tile(t, tm, tn);
+        // column-major over the trapezoid: column tn holds rows tn .. nr-1
+        int u = t;
+        tn = 0;
+        while (u >= nr - tn) {
+          u -= nr - tn;
+          ++tn;
+        }
+        tm = tn + u;
         T.b = panel + int64_t(tn) * NB * lda; T.ldb = lda; T.bt = true;
         T.d = trail + int64_t(tm) * NB * lda + tn * NB;
       } else {
@@ -645,13 +675,16 @@ __global__ void __launch_bounds__(GM_THREADS, 2) k_factor_persistent(FactorArgs 
       T.acc = true;
       return T;
     };
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0 && k + 1 < a.ke) {
       run_tiles64(0, 1, 1, phase_b, sm);     // the next diagonal block first
       diag_factor(a.A, lda, k0 + NB, a.T + size_t(k + 1) * NB * NB, a.status, sm);
     }
     const int workers = nw > 1 ? nw - 1 : 1;
     const int first = nw > 1 ? rank - 1 : 0;
-    if (works && (nw == 1 || blockIdx.x > 0)) run_tiles64(1 + first, workers, n_total, phase_b, sm);
+    // without a lookahead (the last step of the launch) the workers start at tile 0
+    const int t_lo = (k + 1 < a.ke) ? 1 : 0;
+    if (works && (nw == 1 || blockIdx.x > 0))
+      run_tiles64(t_lo + first, workers, n_total, phase_b, sm);
     if (!grid_barrier(a, epoch)) return;
   }
 }
@@ -665,6 +698,42 @@ gptq_status selftest_grid_barrier(cudaStream_t st, int32_t* status) {
   GPTQ_CUDA(cudaMemsetAsync(p, 0, sizeof(g_selftest_slot), st));
   GPTQ_LAUNCH(k_selftest_grid_barrier, 2, 32, 0, st, p, status);
   return GPTQ_OK;
+}
+
+// TF32 hi/lo split (hi: the low 13 mantissa bits cleared) of an M x K block with row
+// stride lds into M x K outputs with row stride ldo.
+__global__ void k_split_rows(const float* src, int64_t lds, int M, int K, float* hi, float* lo,
+                             int ldo) {
+  const int64_t total = int64_t(M) * K;
+  for (int64_t idx = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; idx < total;
+       idx += int64_t(gridDim.x) * blockDim.x) {
+    const int m = int(idx / K), k = int(idx % K);
+    const float v = src[m * lds + k];
+    const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    hi[int64_t(m) * ldo + k] = h;
+    lo[int64_t(m) * ldo + k] = v - h;
+  }
+}
+
+// The same split, transposed: out[n][k] = src[k * lds + n] for a K x N block.
+__global__ void k_split_cols(const float* src, int64_t lds, int K, int N, float* hi, float* lo,
+                             int ldo) {
+  __shared__ float tile[32][33];
+  const int k0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int k = k0 + i, n = n0 + threadIdx.x;
+    tile[i][threadIdx.x] = (k < K && n < N) ? src[k * lds + n] : 0.f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int n = n0 + i, k = k0 + threadIdx.x;
+    if (n < N && k < K) {
+      const float v = tile[threadIdx.x][i];
+      const float h = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+      hi[int64_t(n) * ldo + k] = h;
+      lo[int64_t(n) * ldo + k] = v - h;
+    }
+  }
 }
 
 // U[a][b] = Minv[C-1-a][C-1-b] for a <= b, 0 below the diagonal.
@@ -698,11 +767,12 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
   GPTQ_LAUNCH(k_gather_rev, grid_for(int64_t(Cp) * Cp), 256, 0, st, H, C, Cp, perm, L.lam, L.A,
               L.Bx);
   // Blocked right-looking Cholesky of A interleaved with the blocked forward
-  // substitution that turns Bx = I into M^-1, in one persistent cooperative launch.
+  // substitution that turns Bx = I into M^-1, in persistent cooperative launches:
+  // one for everything, or, above OUTER_MIN_COLS, one per outer panel of
+  // OUTER_BLOCKS steps followed by the outer panel's update of the rest on the
+  // tensor cores.
   unsigned* bar = reinterpret_cast<unsigned*>(reinterpret_cast<char*>(L.lam) + 64);
   int* abort_flag = reinterpret_cast<int*>(reinterpret_cast<char*>(L.lam) + 128);
-  GPTQ_CUDA(cudaMemsetAsync(reinterpret_cast<char*>(L.lam) + 64, 0, 128, st));
-  FactorArgs fa{L.A, L.Bx, L.T, Cp, L.nblk, bar, abort_flag, status, L.smid};
   int per_sm = 0;
   GPTQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_factor_persistent,
                                                           GM_THREADS, 0));
@@ -712,10 +782,29 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
   const int nr0 = Cp / NB - 1;
   const int most = std::max(1, std::max(nr0 * (nr0 + 1) / 2 + nr0, nr0 + Cp / NB));
   const int grid = std::min(std::min(std::min(per_sm, 2) * sms, most + 1), MAX_FACTOR_GRID);
-  void* args[] = {&fa};
-  GPTQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_factor_persistent), dim3(grid),
-                                        dim3(GM_THREADS), args, 0, st));
-  note_launch();
+  const int per = outer_path(Cp) ? OUTER_BLOCKS : L.nblk;
+  for (int ob = 0; ob < L.nblk; ob += per) {
+    const int oe = std::min(ob + per, L.nblk);
+    GPTQ_CUDA(cudaMemsetAsync(reinterpret_cast<char*>(L.lam) + 64, 0, 128, st));
+    FactorArgs fa{L.A, L.Bx, L.T, Cp, L.nblk, bar, abort_flag, status, L.smid, ob, oe, oe};
+    void* args[] = {&fa};
+    GPTQ_CUDA(cudaLaunchCooperativeKernel(reinterpret_cast<void*>(k_factor_persistent),
+                                          dim3(grid), dim3(GM_THREADS), args, 0, st));
+    note_launch();
+    if (oe >= L.nblk) break;
+    // the outer panel L_b = A[oend:, o0:oend] updates the rest:
+    //   A[oend:, oend:] -= L_b L_b^T    and    Bx[oend:, :oend] -= L_b M^-1[o0:oend, :oend]
+    const int o0 = ob * NB, oend = oe * NB, K = oend - o0, Mb = Cp - oend;
+    GPTQ_LAUNCH(k_split_rows, grid_for(int64_t(Mb) * K), 256, 0, st,
+                L.A + int64_t(oend) * Cp + o0, int64_t(Cp), Mb, K, L.Lh, L.Ll, OUTER_K);
+    GPTQ_TRY(gemm3_tf32(st, L.A + int64_t(oend) * Cp + oend, Cp, Mb, 0, Mb, K, L.Lh, L.Ll,
+                        OUTER_K, 0, L.Lh, L.Ll, OUTER_K, Mb, 0, true, status));
+    dim3 sg((oend + 31) / 32, (K + 31) / 32), sb(32, 8);
+    GPTQ_LAUNCH(k_split_cols, sg, sb, 0, st, L.Bx + int64_t(o0) * Cp, int64_t(Cp), K, oend, L.Mh,
+                L.Ml, OUTER_K);
+    GPTQ_TRY(gemm3_tf32(st, L.Bx + int64_t(oend) * Cp, Cp, Mb, 0, oend, K, L.Lh, L.Ll, OUTER_K, 0,
+                        L.Mh, L.Ml, OUTER_K, oend, 0, false, status));
+  }
   GPTQ_LAUNCH(k_write_u, grid_for(int64_t(C) * C), 256, 0, st, L.Bx, Cp, C, U);
   return GPTQ_OK;
 }

@@ -445,12 +445,14 @@ static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R,
     ce = cudaEventRecord(swept, st);
     if (ce == cudaSuccess) ce = cudaStreamWaitEvent(side, swept, 0);
     if (ce != cudaSuccess) break;
+    // W[:, e:cend] -= Err[:, slot window] * U[panel rows, e:cend], with U read as its
+    // transposed split Ut[n][k] = U[k][n]
     if (lvl1)
-      err = trailing_update_tc(side, L.Wk, R, C, i0, SW_B, e1, c1, L.Ehi, L.Elo, SW_LDERR,
-                               slot * SW_B, L.Uhi, L.Ulo, status);
+      err = gemm3_tf32(side, L.Wk, C, R, e1, c1, SW_B, L.Ehi, L.Elo, SW_LDERR, slot * SW_B,
+                       L.Uhi, L.Ulo, C, C, i0, false, status);
     if (err == GPTQ_OK && lvl2)
-      err = trailing_update_tc(side, L.Wk, R, C, S0, S_end - S0, e2, C, L.Ehi, L.Elo, SW_LDERR,
-                               ((p / per) % 2) * SW_B2, L.Uhi, L.Ulo, status);
+      err = gemm3_tf32(side, L.Wk, C, R, e2, C, S_end - S0, L.Ehi, L.Elo, SW_LDERR,
+                       ((p / per) % 2) * SW_B2, L.Uhi, L.Ulo, C, C, S0, false, status);
     if (err != GPTQ_OK) break;
     ce = cudaEventRecord(ev[1 + b], side);
     upd[b] = ce == cudaSuccess;

@@ -37,7 +37,8 @@ _DT = {torch.float32: GPTQ_F32, torch.float16: GPTQ_F16, torch.bfloat16: GPTQ_BF
 # every symbol include/gptq.h declares
 EXPORTS = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare",
            "gptq_quantize_layer", "gptq_pack", "gptq_status_string", "gptq_launch_count",
-           "gptq_last_error", "gptq_prepare_static", "gptq_selftest_timeout")
+           "gptq_last_error", "gptq_prepare_static", "gptq_selftest_timeout",
+           "gptq_repack_sweep_order", "gptq_dequant_matmul", "gptq_debug_set_wait_limit")
 GPTQ_SELFTEST_MBARRIER, GPTQ_SELFTEST_GRID_BARRIER = 0, 1
 
 GPTQ_STATIC_MAX_COLS = 1024
@@ -96,6 +97,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.gptq_selftest_timeout.restype = i32
     lib.gptq_last_error.argtypes = []
     lib.gptq_last_error.restype = ctypes.c_char_p
+    lib.gptq_repack_sweep_order.argtypes = [vp, i64, i64, i32, vp, vp, vp]
+    lib.gptq_repack_sweep_order.restype = i32
+    lib.gptq_dequant_matmul.argtypes = [vp, i32, i64, i64, i64, vp, vp, vp, i32, i32, vp, vp,
+                                        i64, i32, vp]
+    lib.gptq_dequant_matmul.restype = i32
+    lib.gptq_debug_set_wait_limit.argtypes = [ctypes.c_uint32]
+    lib.gptq_debug_set_wait_limit.restype = ctypes.c_uint32
     _lib = lib
     return lib
 
@@ -259,12 +267,61 @@ def gptq_selftest_timeout(which: int, status: torch.Tensor, stream=None) -> None
            "gptq_selftest_timeout")
 
 
+def gptq_debug_set_wait_limit(polls: int) -> int:
+    """Polls after which a tensor-core pipeline wait gives up (0 = the default);
+    returns the previous limit.  For tests of the timeout path."""
+    return int(load_library().gptq_debug_set_wait_limit(int(polls)))
+
+
 def gptq_launch_count() -> int:
     return int(load_library().gptq_launch_count())
 
 
 def gptq_last_error() -> str:
     return load_library().gptq_last_error().decode()
+
+
+# --------------------------------------------------------------------------- stored form
+def sweep_words(cols: int, bits: int) -> int:
+    return cols // 32 * bits
+
+
+def gptq_repack_sweep_order(packed, bits, perm, out, stream=None) -> None:
+    """The packed codes (original column order) rewritten in the sweep order perm."""
+    C = perm.shape[0]
+    if C % 32:
+        raise ValueError("cols must be a multiple of 32")
+    R = packed.shape[0]
+    _expect(packed, "packed", (R, packed_words(C, bits)), (torch.int32, torch.uint32))
+    _expect(perm, "perm", (C,), (torch.int32,))
+    _expect(out, "out", (R, sweep_words(C, bits)), (torch.int32, torch.uint32))
+    _need_cuda(packed, perm, out)
+    _check(load_library().gptq_repack_sweep_order(_ptr(packed), R, C, int(bits), _ptr(perm),
+                                                  _ptr(out), _stream(stream)),
+           "gptq_repack_sweep_order")
+
+
+def gptq_dequant_matmul(X, qp, scales, zeros, bits, group_size, perm, Y, half_sums=False,
+                        stream=None) -> None:
+    """Y (m x rows fp32) = X (m x cols) Q^T from the sweep-order packed codes."""
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be 2-D with unit column stride")
+    if X.dtype not in _DT:
+        raise ValueError(f"X must be float32, float16 or bfloat16, got {X.dtype}")
+    M, C = X.shape
+    R = qp.shape[0]
+    G = n_groups(C, group_size)
+    _expect(qp, "qp", (R, sweep_words(C, bits)), (torch.int32, torch.uint32))
+    _expect(scales, "scales", (R, G), (torch.float32,))
+    _expect(zeros, "zeros", (R, G), (torch.float32,))
+    if perm is not None:
+        _expect(perm, "perm", (C,), (torch.int32,))
+    _expect(Y, "Y", (M, R), (torch.float32,))
+    _need_cuda(X, qp, scales, zeros, perm, Y)
+    _check(load_library().gptq_dequant_matmul(
+        _ptr(X), _DT[X.dtype], M, C, X.stride(0), _ptr(qp), _ptr(scales), _ptr(zeros), int(bits),
+        int(group_size), _ptr(perm), _ptr(Y), R, int(bool(half_sums)), _stream(stream)),
+        "gptq_dequant_matmul")
 
 
 # --------------------------------------------------------------------------- one layer

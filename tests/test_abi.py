@@ -25,7 +25,7 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = G.load_library()
     names = declared_functions()
-    assert len(names) == 10, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(lib, n), n
     assert sorted(G.EXPORTS) == names

@@ -2,7 +2,8 @@
 
 * Layers that read the same input (q/k/v, gate/up) share one Hessian and one
   factorization: quantize_layers_shared must give exactly what separate
-  quantize_layer calls give.
+  quantize_layer calls give, and every weight of the group must match the
+  float64 oracle on the shared Hessian at the stated tolerances.
 * Round-to-nearest is the sweep with U = I (no error is fed forward): its codes
   must be the oracle's round-to-nearest on the same grids, computed from the
   original weights, except at entries whose x/s is within a hair of a rounding
@@ -17,6 +18,7 @@ import torch
 from oracle import gptq_ref as o
 from post_weight_quantization_20_b200 import gptq as G
 from post_weight_quantization_20_b200 import synthetic as S
+from tests.parity import compare_layer
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -60,6 +62,32 @@ def test_shared_input_group_matches_separate_layers():
         for k, v in (("codes", codes), ("scales", scales), ("zeros", zeros), ("g_idx", g_idx),
                      ("losses", losses)):
             assert torch.equal(getattr(r, k), v), k
+
+
+def test_shared_input_group_matches_oracle():
+    """q/k/v-shaped group (three weights, one input): one Hessian and one factor on the
+    GPU; each weight against the oracle's sweep on the oracle's own float64 Hessian of
+    the same calibration tokens, in the same (given) act-order."""
+    C = 512
+    X = S.gen_activations(5000, C, S.F16, S.ActSpec(outlier_frac=0.02, mix_rank=4), seed=21)
+    Ws = [S.gen_weight(R, C, S.F16, S.WeightSpec(outlier_frac=0.001), seed=30 + R)
+          for R in (160, 96, 64)]
+    H64, n = o.hessian(S.to_f64(X, S.F16))
+    perm = o.act_order_perm(H64)
+    cfg = G.make_config(4, 128, act_order=G.GPTQ_ORDER_GIVEN)
+    out = G.quantize_layers_shared([_dev(W, S.F16) for W in Ws], _dev(X, S.F16), cfg,
+                                   perm=torch.from_numpy(perm.astype(np.int32)).to(DEV))
+    torch.cuda.synchronize()
+    prepared = o.prepare(H64, 0.01, False, perm)
+    for k, (W, r) in enumerate(zip(Ws, out)):
+        gpu = {"codes": r.codes.cpu().numpy().astype(np.int64), "scales": r.scales.cpu().numpy(),
+               "zeros": r.zeros.cpu().numpy(), "losses": r.losses.cpu().numpy(),
+               "g_idx": r.g_idx.cpu().numpy().astype(np.int64)}
+        p, ref = compare_layer(S.to_f64(W, S.F16), H64, n, perm, gpu, 4, 128, False,
+                               prepared=prepared)
+        p.assert_bars(f"shared-input group, weight {k} ({W.shape[0]}x{C})")
+        np.testing.assert_array_equal(r.packed.cpu().numpy().view(np.uint32),
+                                      o.pack(gpu["codes"], 4))
 
 
 def _oracle_rtn(W64, bits, group, sym):

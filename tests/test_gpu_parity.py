@@ -104,7 +104,7 @@ def _prep_gpu(H32, cfg, perm=None):
     return U.cpu().numpy().astype(np.float64), p.cpu().numpy(), int(st.item())
 
 
-@pytest.mark.parametrize("cols", [1, 63, 128, 200, 520, 1600, 2200])
+@pytest.mark.parametrize("cols", [1, 63, 128, 200, 520, 1600, 4200])
 @pytest.mark.parametrize("act", [False, True])
 def test_prepare_matches_oracle(cols, act):
     X = S.gen_activations(4 * cols + 64, cols, S.F32, S.ActSpec(dist="t4", mix_rank=3), seed=cols)
@@ -204,6 +204,10 @@ CASES = [
     ("two-level-1408", 96, 1408, 4000, S.F16, S.F16, 4, 128, False, False, S.ActSpec(mix_rank=6)),
     ("two-level-ragged-2200-act", 64, 2200, 5000, S.BF16, S.BF16, 4, 64, False, True,
      S.ActSpec(mix_rank=8)),
+    # more than 3584 columns: the factorization blocked in 512-column outer panels
+    # whose updates of the rest run on the tensor cores
+    ("outer-blocked-4160-act", 48, 4160, 9000, S.F16, S.F16, 4, 128, False, True,
+     S.ActSpec(mix_rank=6)),
 ]
 
 
