@@ -70,6 +70,19 @@ class NotPositiveDefinite(ArithmeticError):
 # -----------------------------------------------------------------------------
 # step 1: Hessian  [Deep-dive §3.1 step 1], [Deep-dive §2.1]
 # -----------------------------------------------------------------------------
+def _xtx(Xd: np.ndarray) -> np.ndarray:
+    """X^T X by general matrix products over blocks of at most 8192 columns (the
+    symmetric rank-k routine behind a plain X.T @ X fails in OpenBLAS once the
+    result has 2^31 or more entries, e.g. 49152 x 49152)."""
+    C = Xd.shape[1]
+    if C <= 8192:
+        return Xd.T @ Xd
+    G = np.empty((C, C))
+    for j0 in range(0, C, 8192):
+        G[:, j0:j0 + 8192] = Xd.T @ Xd[:, j0:j0 + 8192]
+    return G
+
+
 def hessian_accumulate(H: np.ndarray, n: int, X: np.ndarray):
     """Running-mean update H <- H n/(n+m) + 2/(n+m) X^T X for a chunk X (m x cols).
 
@@ -79,7 +92,7 @@ def hessian_accumulate(H: np.ndarray, n: int, X: np.ndarray):
     if m == 0:
         return H, n
     Xd = np.asarray(X, dtype=np.float64)
-    H = H * (n / (n + m)) + (2.0 / (n + m)) * (Xd.T @ Xd)
+    H = H * (n / (n + m)) + (2.0 / (n + m)) * _xtx(Xd)
     return H, n + m
 
 
@@ -95,7 +108,7 @@ def hessian(X: np.ndarray, chunk: int | None = None):
     for t in range(0, X.shape[0], step):
         Xd = np.asarray(X[t:t + step], dtype=np.float64)
         m = int(Xd.shape[0])
-        G = Xd.T @ Xd
+        G = _xtx(Xd)
         G *= 2.0 / (n + m)
         H *= n / (n + m)
         H += G
@@ -122,6 +135,31 @@ def act_order_perm(H: np.ndarray) -> np.ndarray:
     return np.argsort(-np.diag(H), kind="stable").astype(np.int64)
 
 
+# SciPy's LAPACK here takes 32-bit indices: above this order an n x n matrix has
+# 2^31 or more entries and its routines fail (NumPy's own LAPACK takes 64-bit ones)
+LAPACK32_MAX_ORDER = 46340
+
+
+def _inverse_cholesky_upper_wide(Hp: np.ndarray) -> np.ndarray:
+    """The same route for orders above LAPACK32_MAX_ORDER, with NumPy's 64-bit-index
+    LAPACK: Hp = L L^T, L^-1 by a general inverse, Hp^-1 = L^-T L^-1, U = the upper
+    Cholesky factor of Hp^-1."""
+    try:
+        L = np.linalg.cholesky(Hp)
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e)) from e
+    Linv = np.linalg.inv(L)
+    del L
+    Hinv = _xtx(Linv)
+    del Linv
+    try:
+        Lu = np.linalg.cholesky(Hinv)
+    except np.linalg.LinAlgError as e:
+        raise NotPositiveDefinite(str(e)) from e
+    del Hinv
+    return Lu.T.copy()
+
+
 def inverse_cholesky_upper(Hp: np.ndarray) -> np.ndarray:
     """U upper triangular with positive diagonal and U^T U = Hp^-1.
 
@@ -133,6 +171,8 @@ def inverse_cholesky_upper(Hp: np.ndarray) -> np.ndarray:
     C = Hp.shape[0]
     if C == 0:
         return np.zeros((0, 0))
+    if C > LAPACK32_MAX_ORDER:
+        return _inverse_cholesky_upper_wide(Hp)
     try:
         cf = sla.cho_factor(Hp, lower=True, check_finite=True)
     except (np.linalg.LinAlgError, ValueError) as e:

@@ -64,6 +64,7 @@ class Parity:
     def assert_bars(self, name: str, check_losses: bool = True) -> None:
         """The stated tolerances; the summary goes to the session report first."""
         REPORT.append(f"{name}: {self.summary()}")
+        print(f"{name}: {self.summary()}", flush=True)
         assert self.bad_hints == 0, name
         assert self.code_mismatch == 0, name
         assert self.max_forced_dist <= TIE_TAU, name

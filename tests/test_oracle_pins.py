@@ -485,3 +485,15 @@ def test_packing_density_matches_the_quoted_model_sizes(bits):
         assert o.pack(codes, bits).nbytes == 2 * cols * bits // 8
     assert 175e9 * bits / 8 / 1e9 == pytest.approx({4: 87.5, 3: 65.6}[bits], abs=0.05)
 
+
+
+def test_wide_inverse_factor_route_matches_the_potri_route():
+    """Above 46340 columns the oracle forms U with NumPy's 64-bit-index LAPACK (a
+    general inverse of the Cholesky factor) instead of SciPy's potri; both routes give
+    the same U, checked here at a small order, and it satisfies U^T U Hp = I."""
+    Hp = gen_spd(200, seed=11, cond=1e4)
+    U1 = o.inverse_cholesky_upper(Hp)
+    U2 = o._inverse_cholesky_upper_wide(Hp)
+    assert np.allclose(np.tril(U2, -1), 0.0) and np.all(np.diag(U2) > 0)
+    assert np.linalg.norm(U1 - U2) <= 1e-10 * np.linalg.norm(U1)
+    assert np.abs(U2.T @ U2 @ Hp - np.eye(200)).max() < 1e-8
