@@ -43,11 +43,16 @@ from post_weight_quantization_20_b200.workloads import WORKLOADS  # noqa: E402
 
 METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per Hessian launch from an ncu capture of the current
-# kernel, as bytes per token at the captured column count (a small case, scaled
-# to the bench's launch by the token count), or None when the kernel has changed
-# since its last capture.
-HESSIAN_TRAFFIC = None
+# DRAM bytes (read + write) of the Hessian launch at the given column count, per
+# calibration token, or None when the kernel has changed since the counters were
+# taken.  Estimated from two ncu captures at 24576 columns (8192 and 16384 tokens):
+# X's re-reads per flop at 16384 tokens (1.066 GB per TFLOP, the streaming rate)
+# times the launch's 6.33e14 flop, plus H's triangle read and written once
+# (2 x 4.83 GB): 685 GB per 262144-token launch.
+HESSIAN_TRAFFIC = {"cols": 49152, "bytes_per_token": 685e9 / 262144,
+                   "how": "estimate scaled from ncu captures at 24576 columns, 8192 and 16384 "
+                          "tokens (X re-reads per flop at the streaming rate, plus the H "
+                          "triangle read and written once)"}
 
 
 def load_peaks():
@@ -422,7 +427,8 @@ def run_ours(args, rank, world, local_rank):
     n_layers = len(layers) * world
     peaks = load_peaks()
     achieved = hess_flop / (hess_ms * 1e-3) / 1e12 if hess_ms > 0 else None
-    peak = float(peaks["bf16_tflops"])
+    # the Hessian runs inside a step of seconds at the power cap: the sustained peak
+    peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
     traffic = None
     if HESSIAN_TRAFFIC:
         toks = [m for _, _, m, C in hess_ev if C == HESSIAN_TRAFFIC["cols"]]
@@ -448,11 +454,13 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "hessian accumulate (X^T X)",
                      "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                     "traffic_scope": (f"bytes per C={HESSIAN_TRAFFIC['cols']} launch, from an "
-                                       "ncu capture of a smaller token count scaled by tokens")
+                     "traffic_scope": (f"bytes per C={HESSIAN_TRAFFIC['cols']} launch: "
+                                       f"{HESSIAN_TRAFFIC['how']}")
                      if traffic is not None else
                      "null: the kernel changed after its last ncu capture",
-                     "peak_source": f"{peaks['source']} bf16 dense burst"},
+                     "peak_source": (f"{peaks['source']} bf16 dense, sustained (a seconds-long "
+                                     f"loop at the power cap), as the Hessian runs inside a "
+                                     f"step of seconds; burst {float(peaks['bf16_tflops']):g}")},
         "e2e": {"value": e2e_ms / n_layers_rank, "unit": "ms", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h)},
         "stored_form": stored,
@@ -705,6 +713,21 @@ def run_op(args):
         def run():
             G.gptq_prepare(H, cfg, U, perm, wsp, status)
         work = f"{2.0 * C ** 3 / 3e12:.4f} TFLOP per call (2/3 C^3)"
+    elif args.op == "dequant":
+        # the stored form's product for args.tokens (<= 8) decode tokens on random codes
+        Gn = G.n_groups(C, cfg.group_size)
+        words = torch.randint(-2 ** 31, 2 ** 31 - 1, (R, G.sweep_words(C, cfg.bits)),
+                              dtype=torch.int32, device=dev, generator=gen)
+        sc = torch.rand(R, Gn, device=dev, generator=gen) * 0.01
+        ze = torch.randint(0, 2 ** cfg.bits, (R, Gn), device=dev, generator=gen).float()
+        pm = torch.randperm(C, device=dev, generator=gen).int()
+        x = torch.randn(min(T, 8), C, device=dev, generator=gen).half()
+        y = torch.empty(x.shape[0], R, device=dev)
+
+        def run():
+            G.gptq_dequant_matmul(x, words, sc, ze, cfg.bits, cfg.group_size, pm, y)
+        nbytes = R * C * cfg.bits // 8 + R * Gn * 8 + x.numel() * 2 + y.numel() * 4
+        work = f"{nbytes / 1e6:.1f} MB of codes, grids, tokens and outputs per call"
     elif args.op == "quantize":
         G.gptq_prepare(H, cfg, U, perm, wsp, status)
         Gn = G.n_groups(C, cfg.group_size)
@@ -749,7 +772,7 @@ def main():
     ap.add_argument("--workload", default="opt175b", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", default="step", choices=["step", "hessian", "prepare", "quantize",
-                                                     "layer"])
+                                                     "layer", "dequant"])
     ap.add_argument("--rows", type=int, default=768)
     ap.add_argument("--cols", type=int, default=3072)
     ap.add_argument("--tokens", type=int, default=16384)

@@ -23,8 +23,9 @@ constexpr int KC = 2048;          // columns of X staged per chunk
 constexpr int UNITS = KC / 32;    // 64 units per chunk
 constexpr int XLD = 36;           // floats per staged unit (32 + 4 pad: conflict-free float4)
 constexpr int WARPS = 8;
-constexpr int RW = 2;             // rows per warp
-constexpr int ROWS = WARPS * RW;  // rows per CTA
+constexpr int RW = 4;             // rows per warp
+constexpr int ROWS = WARPS * RW;  // rows per CTA: the staged X block serves 32 rows
+constexpr int UPL = UNITS / 32;   // units of a chunk per lane
 
 
 // code i (0..31) of a unit held in words w[0..B-1]
@@ -75,6 +76,24 @@ k_dq_gemv(const void* __restrict__ X, int xdt, int64_t ldx, int M, const uint32_
 
   for (int c0 = 0; c0 < C; c0 += KC) {
     const int nu = min(KC, C - c0) >> 5;
+    // all of the lane's code words of this chunk (RW rows x UPL units) are loaded
+    // first, so that they are in flight while X is staged
+    uint32_t w[RW][UPL][B];
+#pragma unroll
+    for (int a = 0; a < RW; ++a) {
+      const int r = r0 + a;
+      const uint32_t* row = Qp + int64_t(r) * words + int64_t(c0 >> 5) * B;
+#pragma unroll
+      for (int j = 0; j < UPL; ++j) {
+        const int u = lane + 32 * j;
+        if (r < R && u < nu) {
+          load_unit<B>(row + int64_t(u) * B, w[a][j]);
+        } else {
+#pragma unroll
+          for (int k = 0; k < B; ++k) w[a][j][k] = 0u;
+        }
+      }
+    }
     __syncthreads();                               // the previous chunk is consumed
     for (int e = threadIdx.x; e < MT * nu * 32; e += blockDim.x) {
       const int m = e / (nu * 32), j = e - m * nu * 32;
@@ -97,10 +116,10 @@ k_dq_gemv(const void* __restrict__ X, int xdt, int64_t ldx, int M, const uint32_
     for (int a = 0; a < RW; ++a) {
       const int r = r0 + a;
       if (r >= R) break;
-      const uint32_t* row = Qp + int64_t(r) * words + int64_t(c0 >> 5) * B;
-      for (int u = lane; u < nu; u += 32) {
-        uint32_t w[B];
-        load_unit<B>(row + int64_t(u) * B, w);
+#pragma unroll
+      for (int j = 0; j < UPL; ++j) {
+        const int u = lane + 32 * j;
+        if (u >= nu) break;
         const int g = gshift < 0 ? 0 : ((c0 + 32 * u) >> gshift);
         const float s = __ldg(scales + int64_t(r) * G + g);
         const float z = __ldg(zeros + int64_t(r) * G + g);
@@ -111,7 +130,9 @@ k_dq_gemv(const void* __restrict__ X, int xdt, int64_t ldx, int M, const uint32_
         for (int i4 = 0; i4 < 32; i4 += 4) {
           float cf[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) cf[q] = float(field<B>(w, i4 + q));
+          // code -> float without I2F: 2^23 + c as bits, minus 2^23 (exact for c < 2^23)
+          for (int q = 0; q < 4; ++q)
+            cf[q] = __int_as_float(0x4B000000u | field<B>(w[a][j], i4 + q)) - 8388608.f;
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
             const float4 xv = *reinterpret_cast<const float4*>(xs + (m * UNITS + u) * XLD + i4);

@@ -39,7 +39,7 @@ constexpr int A_BOX = TM * TK * 4;                 // 8 KB: 128 rows x 64 B
 constexpr int B_BOX = 128 * TK * 4;                // 8 KB: 128 N-rows x 64 B
 constexpr int STAGE = 2 * A_BOX + 2 * (TN / 128) * B_BOX;   // 48 KB
 constexpr int STAGES = 4;
-constexpr int SEG_STAGES = 2;                      // stages per TMEM segment (32 K-values)
+constexpr int MAX_SEG = 2;       // stages per TMEM segment: 1 (16 K-values) or 2 (32)
 constexpr int THREADS = 320;
 constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 2 * TN;
@@ -56,6 +56,7 @@ struct Prob {
   int lower;         // skip tiles with no entry on or below the diagonal (n - n_lo <= m)
   int vec;           // D rows 16-byte aligned
   uint32_t wait_limit;   // polls of an mbarrier wait before it gives up
+  int seg;               // stages per TMEM segment (1 .. MAX_SEG)
 };
 
 // t-th tile in grouped order: GROUP_M row tiles, all column tiles, then the next group.
@@ -90,7 +91,7 @@ k_gemm3_tf32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CU
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.ntm * p.ntn;
-  const int nseg = (p.nk + SEG_STAGES - 1) / SEG_STAGES;
+  const int nseg = (p.nk + p.seg - 1) / p.seg;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -156,7 +157,7 @@ k_gemm3_tf32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CU
         tile_of(p, w, tm, tn);
         if (!tile_live(p, tm, tn)) continue;
         for (int sg = 0; sg < nseg && ok; ++sg) {
-          const int s0 = sg * SEG_STAGES, s1 = min(s0 + SEG_STAGES, p.nk);
+          const int s0 = sg * p.seg, s1 = min(s0 + p.seg, p.nk);
           if (!tc::mbar_wait(acc_empty + acc, acc_phase ^ 1u, abort_flag, p.wait_limit)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t d = tmem_base + uint32_t(acc * TN);
@@ -300,7 +301,7 @@ bool encode_k_major(CUtensorMap* m, const float* base, uint64_t ld, uint64_t row
 gptq_status gemm3_tf32(cudaStream_t st, float* D, int64_t ldd, int M, int n_lo, int n_hi, int K,
                        const float* Ahi, const float* Alo, int lda, int a_k0, const float* Bhi,
                        const float* Blo, int ldb, int b_rows, int b_k0, bool lower,
-                       int32_t* status) {
+                       int32_t* status, int seg_k) {
   if (M <= 0 || n_hi <= n_lo || K <= 0) return GPTQ_OK;
   // K windows start on 16-byte boundaries (TMA x coordinate) and are whole stages
   if (K % TK || a_k0 % 4 || b_k0 % 4 || a_k0 + K > lda || b_k0 + K > ldb || n_lo < 0 ||
@@ -327,6 +328,7 @@ gptq_status gemm3_tf32(cudaStream_t st, float* D, int64_t ldd, int M, int n_lo, 
   p.lower = lower ? 1 : 0;
   p.vec = ((ldd & 3) == 0 && (reinterpret_cast<uintptr_t>(D) & 15) == 0) ? 1 : 0;
   p.wait_limit = pipeline_wait_limit();
+  p.seg = std::max(1, std::min(MAX_SEG, seg_k / TK));
   int64_t live = int64_t(p.ntm) * p.ntn;
   if (lower) {
     live = 0;

@@ -368,9 +368,16 @@ def _on(stream):
     return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
 
 
-def _hessian(X, C: int, dev, status, chunk_tokens, stream):
-    H = torch.empty(C, C, dtype=torch.float32, device=dev)
-    n = 0
+def _hessian(X, C: int, dev, status, chunk_tokens, stream, n_start: int = 0):
+    """H of the tokens of X (a tensor or an iterable of chunks).  n_start > 0 starts
+    the running mean as if n_start tokens of a zero Hessian had been seen already,
+    so that the result is (2 / (n_start + n)) X^T X: a share of a Hessian whose
+    tokens are split over several callers."""
+    if n_start > 0:
+        H = torch.zeros(C, C, dtype=torch.float32, device=dev)
+    else:
+        H = torch.empty(C, C, dtype=torch.float32, device=dev)
+    n = int(n_start)
     chunks = [X] if isinstance(X, torch.Tensor) else X
     for Xc in chunks:
         if chunk_tokens:

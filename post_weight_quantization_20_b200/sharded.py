@@ -2,9 +2,11 @@
 
 The layer shards two ways (GPTQ量化算法深度解析 §3.1 step 1 and §2.4):
 
-* tokens: H = 2/N sum_t x_t x_t^T is a mean over the calibration tokens, so rank r
-  accumulates the Hessian H_r of its own n_r tokens with the library, and one
-  all-reduce of (n_r / N) H_r gives the layer's H on every rank;
+* tokens: H = 2/N sum_t x_t x_t^T is a mean over the calibration tokens.  The
+  ranks first add up their token counts (N); rank r then accumulates its share
+  (2/N) sum_{t in r} x_t x_t^T with the library, its running mean started at the
+  N - n_r tokens of the other ranks, and one all-reduce (a sum) of the shares
+  gives the layer's H on every rank;
 * rows: given U and the column order, the compensation runs along each row only,
   so every rank sweeps its own rows of W; the per-column losses (sums over rows)
   take one more all-reduce.
@@ -37,20 +39,23 @@ def row_range(rows: int, world: int, rank: int) -> tuple[int, int]:
     return r0, r0 + base + (1 if rank < extra else 0)
 
 
-def combine_hessians(H: torch.Tensor, n_local: int, group=None) -> int:
-    """In place: H <- sum_r (n_r / N) H_r over the ranks of `group`, N = sum_r n_r.
-    H holds this rank's running-mean Hessian of n_local tokens (upper triangle; a
-    rank with no tokens contributes zeros whatever H holds).  Returns N."""
-    n = torch.tensor([int(n_local)], dtype=torch.int64, device=H.device)
+def token_count(X_local) -> int:
+    """Tokens of a rank's calibration input: a tokens x cols tensor or a sequence of
+    such chunks (the count is needed before the first accumulation)."""
+    if isinstance(X_local, torch.Tensor):
+        return int(X_local.shape[0])
+    if isinstance(X_local, (list, tuple)):
+        return sum(int(x.shape[0]) for x in X_local)
+    raise TypeError("X_local must be a tensor or a list / tuple of chunks")
+
+
+def total_tokens(n_local: int, device, group=None) -> int:
+    """The number of calibration tokens over the ranks of `group`."""
+    n = torch.tensor([int(n_local)], dtype=torch.int64, device=device)
     dist.all_reduce(n, group=group)
     total = int(n.item())
     if total <= 0:
         raise ValueError("no calibration tokens on any rank")
-    if n_local == 0:
-        H.zero_()
-    else:
-        H.mul_(float(n_local) / float(total))
-    dist.all_reduce(H, group=group)
     return total
 
 
@@ -64,16 +69,19 @@ def quantize_layer_sharded(W_rows: torch.Tensor, X_local, cfg: G.gptq_config, gr
                            perm: torch.Tensor | None = None, chunk_tokens: int | None = None,
                            stream=None, check: bool = True) -> G.LayerResult:
     """Quantize this rank's rows W_rows (rows_r x cols) of a layer whose calibration
-    tokens are split over the ranks (X_local: this rank's tokens x cols, or an
-    iterable of such chunks; it may hold no tokens).  Returns this rank's rows of
+    tokens are split over the ranks (X_local: this rank's tokens x cols, or a list of
+    such chunks; it may hold no tokens).  Returns this rank's rows of
     codes, scales, zeros and packed words, and the layer's g_idx, order, H, U, total
     token count and per-column losses summed over all ranks' rows."""
     dev = W_rows.device
     C = W_rows.shape[1]
     with G._on(stream):
         status = torch.zeros(1, dtype=torch.int32, device=dev)
-        H, n = G._hessian(X_local, C, dev, status, chunk_tokens, stream)
-        total = combine_hessians(H, n, group)
+        n_local = token_count(X_local)
+        total = total_tokens(n_local, dev, group)
+        H, n = G._hessian(X_local, C, dev, status, chunk_tokens, stream,
+                          n_start=total - n_local)
+        dist.all_reduce(H, group=group)       # the sum of the shares: the layer's H
         U, perm = G._factor(H, cfg, perm, W_rows.shape[0], dev, status, stream)
         codes, scales, zeros, g_idx, losses, packed = G._sweep(W_rows, U, perm, cfg, dev, status,
                                                                stream)

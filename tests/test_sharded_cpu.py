@@ -2,8 +2,9 @@
 
 Calibration tokens are split unevenly over two or three ranks (some cases give a
 rank no tokens) and the rows of W are split by row_range.  The library's three steps are
-replaced on CPU by stand-ins: the Hessian of the rank's tokens in torch, and the
-oracle's factorization and sweep.  What is checked is the sharding itself:
+replaced on CPU by stand-ins: the running-mean Hessian of the rank's tokens in
+torch (started, like the library's, at the other ranks' token count on a zero H),
+and the oracle's factorization and sweep.  What is checked is the sharding itself:
   * the combined H equals the Hessian of all tokens and is bitwise the same on
     both ranks (each rank factors its own copy);
   * the token count is the total over ranks;
@@ -41,13 +42,19 @@ def _free_port():
 
 def _cpu_steps(G, o):
     """CPU stand-ins for the library's Hessian, factorization and sweep."""
-    def hessian(X, C, dev, status, chunk_tokens, stream):
+    def hessian(X, C, dev, status, chunk_tokens, stream, n_start=0):
+        # the library's running mean, started at n_start tokens of a zero Hessian
         X = X.double()
-        n = X.shape[0]
-        H = torch.full((C, C), float("nan"), dtype=torch.float32)   # like torch.empty
-        if n:
-            H = (2.0 / n * (X.T @ X)).float()
-        return H, n
+        m = X.shape[0]
+        if n_start > 0:
+            H = torch.zeros((C, C), dtype=torch.float64)
+        else:
+            H = torch.full((C, C), float("nan"), dtype=torch.float64)   # like torch.empty
+        if m:
+            # with no tokens seen, the first chunk overwrites H (the library's rule)
+            prev = H * (n_start / (n_start + m)) if n_start > 0 else 0.0
+            H = prev + (2.0 / (n_start + m)) * (X.T @ X)
+        return H.float(), n_start + m
 
     def factor(H, cfg, perm, rows, dev, status, stream):
         p, _, U = o.prepare(H.double().numpy(), cfg.damp, cfg.act_order == 1)
