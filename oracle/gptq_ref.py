@@ -136,28 +136,82 @@ def act_order_perm(H: np.ndarray) -> np.ndarray:
 
 
 # SciPy's LAPACK here takes 32-bit indices: above this order an n x n matrix has
-# 2^31 or more entries and its routines fail (NumPy's own LAPACK takes 64-bit ones)
+# 2^31 or more entries and its routines fail; NumPy's own (64-bit) LAPACK and
+# symmetric products crash on matrices that large (49152^2).  Above it the
+# factorizations run as the textbook block algorithms over WIDE_BLOCK columns, each
+# block step a LAPACK call of order WIDE_BLOCK or a general matrix product.
 LAPACK32_MAX_ORDER = 46340
+WIDE_BLOCK = 8192
 
 
-def _inverse_cholesky_upper_wide(Hp: np.ndarray) -> np.ndarray:
-    """The same route for orders above LAPACK32_MAX_ORDER, with NumPy's 64-bit-index
-    LAPACK: Hp = L L^T, L^-1 by a general inverse, Hp^-1 = L^-T L^-1, U = the upper
-    Cholesky factor of Hp^-1."""
-    try:
-        L = np.linalg.cholesky(Hp)
-    except np.linalg.LinAlgError as e:
-        raise NotPositiveDefinite(str(e)) from e
-    Linv = np.linalg.inv(L)
+def _cholesky_lower_blocked(A: np.ndarray, nb: int = WIDE_BLOCK, overwrite: bool = False):
+    """Lower L with L L^T = A (its lower triangle is read) by the right-looking block
+    Cholesky algorithm: for each diagonal block k, L_kk = chol(A_kk); the blocks
+    below it L_ik = A_ik L_kk^-T; then A_ij -= L_ik L_jk^T on the trailing lower
+    blocks.  With overwrite, A's storage becomes L."""
+    n = A.shape[0]
+    L = A if overwrite else np.array(A, dtype=np.float64, copy=True)
+    for k0 in range(0, n, nb):
+        k1 = min(k0 + nb, n)
+        try:
+            Lkk = sla.cholesky(L[k0:k1, k0:k1], lower=True, check_finite=True)
+        except (np.linalg.LinAlgError, ValueError) as e:
+            raise NotPositiveDefinite(str(e)) from e
+        L[k0:k1, k0:k1] = Lkk
+        L[k0:k1, k1:] = 0.0
+        if k1 == n:
+            break
+        P = sla.solve_triangular(Lkk, L[k1:, k0:k1].T, lower=True, check_finite=False).T
+        L[k1:, k0:k1] = P
+        for j0 in range(k1, n, nb):
+            j1 = min(j0 + nb, n)
+            L[j0:, j0:j1] -= P[j0 - k1:] @ P[j0 - k1:j1 - k1].T
+    return L
+
+
+def _tri_inverse_lower_blocked(L: np.ndarray, nb: int = WIDE_BLOCK) -> np.ndarray:
+    """L^-1 for lower triangular L by block forward substitution on the identity:
+    X_jj = L_jj^-1 and, below it, X_ij = -L_ii^-1 sum_{j <= k < i} L_ik X_kj."""
+    n = L.shape[0]
+    X = np.zeros((n, n))
+    for j0 in range(0, n, nb):
+        j1 = min(j0 + nb, n)
+        for i0 in range(j0, n, nb):
+            i1 = min(i0 + nb, n)
+            if i0 == j0:
+                rhs = np.eye(j1 - j0)
+            else:
+                rhs = -(L[i0:i1, j0:i0] @ X[j0:i0, j0:j1])
+            X[i0:i1, j0:j1] = sla.solve_triangular(L[i0:i1, i0:i1], rhs, lower=True,
+                                                    check_finite=False)
+    return X
+
+
+def _lower_gram_of_lower(X: np.ndarray, nb: int = WIDE_BLOCK) -> np.ndarray:
+    """The lower triangle (by block columns; zeros above them) of X^T X for lower
+    triangular X: entry (i, j) sums X[k, i] X[k, j] over k >= j, since X[k, j] = 0
+    for k < j, so block column j0 .. j1-1 takes only rows k >= j0."""
+    n = X.shape[0]
+    G = np.zeros((n, n))
+    for j0 in range(0, n, nb):
+        j1 = min(j0 + nb, n)
+        G[j0:, j0:j1] = X[j0:, j0:].T @ X[j0:, j0:j1]
+    return G
+
+
+def _inverse_cholesky_upper_wide(Hp: np.ndarray, nb: int = WIDE_BLOCK) -> np.ndarray:
+    """The same route for orders above LAPACK32_MAX_ORDER, on the block algorithms:
+    Hp = L L^T, L^-1, Hp^-1 = L^-T L^-1 (its lower triangle, all the factorization
+    reads), U = the upper Cholesky factor of Hp^-1."""
+    L = _cholesky_lower_blocked(Hp, nb)
+    Linv = _tri_inverse_lower_blocked(L, nb)
     del L
-    Hinv = _xtx(Linv)
+    Hinv = _lower_gram_of_lower(Linv, nb)
     del Linv
-    try:
-        Lu = np.linalg.cholesky(Hinv)
-    except np.linalg.LinAlgError as e:
-        raise NotPositiveDefinite(str(e)) from e
-    del Hinv
-    return Lu.T.copy()
+    Lu = _cholesky_lower_blocked(Hinv, nb, overwrite=True)
+    U = np.ascontiguousarray(Lu.T)
+    del Lu, Hinv
+    return U
 
 
 def inverse_cholesky_upper(Hp: np.ndarray) -> np.ndarray:

@@ -487,13 +487,44 @@ def test_packing_density_matches_the_quoted_model_sizes(bits):
 
 
 
+def test_block_cholesky_matches_lapack():
+    """The block Cholesky used above 46340 columns against LAPACK's unblocked one, with
+    blocks of 64 on an order of 300 (a ragged last block)."""
+    A = gen_spd(300, seed=12, cond=1e5)
+    L = o._cholesky_lower_blocked(A, nb=64)
+    assert np.allclose(np.triu(L, 1), 0.0)
+    assert np.linalg.norm(L - np.linalg.cholesky(A)) <= 1e-12 * np.linalg.norm(L)
+    # a block that is not positive definite is reported
+    B = A.copy()
+    B[200, 200] = -1.0
+    with pytest.raises(o.NotPositiveDefinite):
+        o._cholesky_lower_blocked(B, nb=64)
+
+
+def test_block_triangular_inverse_matches_a_general_inverse():
+    L = np.linalg.cholesky(gen_spd(300, seed=13, cond=1e4))
+    X = o._tri_inverse_lower_blocked(L, nb=64)
+    assert np.allclose(np.triu(X, 1), 0.0)
+    assert np.abs(X @ L - np.eye(300)).max() < 1e-10
+    assert np.linalg.norm(X - np.linalg.inv(L)) <= 1e-10 * np.linalg.norm(X)
+
+
+def test_lower_gram_of_a_lower_triangular_matrix():
+    X = np.tril(np.random.default_rng(14).standard_normal((300, 300)))
+    G = o._lower_gram_of_lower(X, nb=64)
+    full = X.T @ X
+    for j0 in range(0, 300, 64):       # block columns: rows from the block's first column
+        np.testing.assert_allclose(G[j0:, j0:j0 + 64], full[j0:, j0:j0 + 64], rtol=1e-12, atol=1e-12)
+    assert np.all(G[np.triu_indices(300, 64)] == 0.0)
+
+
 def test_wide_inverse_factor_route_matches_the_potri_route():
-    """Above 46340 columns the oracle forms U with NumPy's 64-bit-index LAPACK (a
-    general inverse of the Cholesky factor) instead of SciPy's potri; both routes give
-    the same U, checked here at a small order, and it satisfies U^T U Hp = I."""
+    """Above 46340 columns the oracle forms U on the block algorithms instead of
+    SciPy's potri; both routes give the same U, checked here at a small order with
+    blocks of 64, and it satisfies U^T U Hp = I."""
     Hp = gen_spd(200, seed=11, cond=1e4)
     U1 = o.inverse_cholesky_upper(Hp)
-    U2 = o._inverse_cholesky_upper_wide(Hp)
+    U2 = o._inverse_cholesky_upper_wide(Hp, nb=64)
     assert np.allclose(np.tril(U2, -1), 0.0) and np.all(np.diag(U2) > 0)
     assert np.linalg.norm(U1 - U2) <= 1e-10 * np.linalg.norm(U1)
     assert np.abs(U2.T @ U2 @ Hp - np.eye(200)).max() < 1e-8
