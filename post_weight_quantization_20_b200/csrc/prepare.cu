@@ -159,6 +159,74 @@ __global__ void k_gather_rev(const float* H, int C, int Cp, const int32_t* perm,
   }
 }
 
+// The same gather in three coalesced passes, for C up to the columns whose row fits
+// in shared memory (the one-pass gather above reads H column-scattered, ~10x its bytes):
+//   1. S = H with its lower triangle filled from the upper (32 x 32 tiles, the lower
+//      ones transposed through shared memory), into the Bx buffer;
+//   2. A[a][:] = S[i][perm[C-1-b]] with i = perm[C-1-a]: one CTA per row a stages
+//      row i of S in shared memory and writes row a of A in order (lambda on the
+//      diagonal, identity padding);
+//   3. Bx = I.
+constexpr int GATHER_SMEM_MAX_COLS = 56 * 1024;
+
+__global__ void k_sym_full(const float* H, int C, float* S, int lds) {
+  __shared__ float t[32][33];
+  const int bi = blockIdx.y, bj = blockIdx.x;       // output tile (rows bi, cols bj)
+  const int tx = threadIdx.x, ty = threadIdx.y;      // 32 x 8
+  const int si = bi <= bj ? bi : bj, sj = bi <= bj ? bj : bi;   // the upper source tile
+#pragma unroll
+  for (int k = 0; k < 32; k += 8) {
+    const int r = si * 32 + ty + k, c = sj * 32 + tx;
+    t[ty + k][tx] = (r < C && c < C) ? H[int64_t(r) * C + c] : 0.f;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 32; k += 8) {
+    const int rr = ty + k, cc = tx;                  // position inside the output tile
+    const int r = bi * 32 + rr, c = bj * 32 + cc;
+    if (r >= C || c >= C) continue;
+    float v;
+    if (bi < bj) v = t[rr][cc];
+    else if (bi > bj) v = t[cc][rr];
+    else v = rr <= cc ? t[rr][cc] : t[cc][rr];
+    S[int64_t(r) * lds + c] = v;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+k_gather_rows(const float* S, int lds, int C, int Cp, const int32_t* perm, const float* lam,
+              float* A) {
+  extern __shared__ float srow[];
+  const int a = blockIdx.x;
+  float* arow = A + int64_t(a) * Cp;
+  if (a >= C) {
+    for (int b = threadIdx.x; b < Cp; b += blockDim.x) arow[b] = (a == b) ? 1.f : 0.f;
+    return;
+  }
+  int i = perm[C - 1 - a];
+  i = min(max(i, 0), C - 1);
+  const float* src = S + int64_t(i) * lds;
+  for (int b = threadIdx.x; b < C; b += blockDim.x) srow[b] = src[b];
+  __syncthreads();
+  const float l = *lam;
+  for (int b = threadIdx.x; b < Cp; b += blockDim.x) {
+    float v;
+    if (b < C) {
+      int j = perm[C - 1 - b];
+      j = min(max(j, 0), C - 1);
+      v = srow[j] + (a == b ? l : 0.f);
+    } else {
+      v = (a == b) ? 1.f : 0.f;
+    }
+    arow[b] = v;
+  }
+}
+
+__global__ void k_unit_diag(float* Bx, int Cp) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < Cp) Bx[int64_t(i) * Cp + i] = 1.f;
+}
+
 // ---------------------------------------------------------------------------
 // Diagonal blocks: Cholesky factor L of the 64x64 block and T = L^-1 by one CTA
 // holding the block in registers, four columns per step.
@@ -764,8 +832,18 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
     GPTQ_LAUNCH(k_perm_check, pb, 256, 0, st, L.cnt, C, status);
   }
   const int Cp = L.Cp;
-  GPTQ_LAUNCH(k_gather_rev, grid_for(int64_t(Cp) * Cp), 256, 0, st, H, C, Cp, perm, L.lam, L.A,
-              L.Bx);
+  if (C <= GATHER_SMEM_MAX_COLS) {
+    dim3 tg((C + 31) / 32, (C + 31) / 32), tb(32, 8);
+    GPTQ_LAUNCH(k_sym_full, tg, tb, 0, st, H, C, L.Bx, Cp);
+    // the attribute is the largest row any call stages, so concurrent calls agree
+    GPTQ_CUDA(allow_smem(k_gather_rows, GATHER_SMEM_MAX_COLS * 4));
+    GPTQ_LAUNCH(k_gather_rows, Cp, 256, C * 4, st, L.Bx, Cp, C, Cp, perm, L.lam, L.A);
+    GPTQ_CUDA(cudaMemsetAsync(L.Bx, 0, size_t(Cp) * Cp * sizeof(float), st));
+    GPTQ_LAUNCH(k_unit_diag, (Cp + 255) / 256, 256, 0, st, L.Bx, Cp);
+  } else {
+    GPTQ_LAUNCH(k_gather_rev, grid_for(int64_t(Cp) * Cp), 256, 0, st, H, C, Cp, perm, L.lam, L.A,
+                L.Bx);
+  }
   // Blocked right-looking Cholesky of A interleaved with the blocked forward
   // substitution that turns Bx = I into M^-1, in persistent cooperative launches:
   // one for everything, or, above OUTER_MIN_COLS, one per outer panel of
