@@ -45,8 +45,14 @@ METRIC = "ms per linear layer quantized (H+Cholesky+sweep); GEMM TFLOP/s vs B200
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of the Hessian launch at the given column count, per
 # calibration token, or None when the kernel has changed since the counters were
-# taken (the CTA-pair kernel has not been captured yet).
-HESSIAN_TRAFFIC = None
+# taken.  Estimated from two ncu captures of the CTA-pair kernel at 24576 columns
+# (8192 and 16384 tokens): X's re-reads per flop at 16384 tokens (1.99 GB per TFLOP)
+# times the launch's 6.33e14 flop, plus H's triangle read and written once
+# (2 x 4.83 GB): 1271 GB per 262144-token launch.
+HESSIAN_TRAFFIC = {"cols": 49152, "bytes_per_token": 1271e9 / 262144,
+                   "how": "estimate scaled from ncu captures of the CTA-pair kernel at 24576 "
+                          "columns, 8192 and 16384 tokens (X re-reads per flop, plus the H "
+                          "triangle read and written once)"}
 
 
 def load_peaks():
