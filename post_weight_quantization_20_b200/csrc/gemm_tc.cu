@@ -11,16 +11,18 @@
 // Precision.  The tensor core's fp32 accumulation does not round to nearest, so a
 // long chain of MMAs into one TMEM accumulator drifts by about an ulp of the
 // running sum per MMA (over a K = 512 update that made the factor's error five
-// times that of round-to-nearest fp32).  The MMAs therefore accumulate 32 K-values
-// (12 MMAs, two stages) into one of two TMEM buffers, and the epilogue adds each
+// times that of round-to-nearest fp32).  The MMAs therefore accumulate one stage,
+// 32 K-values (12 MMAs), into one of two TMEM buffers, and the epilogue adds each
 // such segment into registers with round-to-nearest fp32 adds while the MMAs fill
 // the other buffer.  At the end of a tile the registers are subtracted from D.
 //
 // Persistent grid of one CTA per SM over 128 x 256 output tiles in grouped order
 // (GROUP_M row tiles per group, so that the tiles in flight together share
 // operand rows in L2).  Per CTA:
-//   warp 0      TMA producer (4-stage ring; a stage is 16 K-values of A hi/lo and
-//               B hi/lo in 64-byte swizzled rows, 48 KB)
+//   warp 0      TMA producer (2-stage ring; a stage is 32 K-values of A hi/lo and
+//               B hi/lo in 128-byte swizzled rows, 96 KB).  Rows of 128 bytes halve
+//               the TMA row requests per byte against 64-byte rows (16 K-values
+//               per stage, four 48 KB stages), which measured 8-10% slower.
 //   warp 1      TMEM allocator and MMA issuer (tcgen05.mma kind::tf32, M=128 N=256 K=8)
 //   warps 2-9   epilogue: two warps per TMEM lane quadrant, 128 columns each
 // Every mbarrier wait is bounded; a wait that gives up sets GPTQ_ERR_TIMEOUT and
@@ -34,12 +36,11 @@ namespace gptq {
 
 namespace {
 
-constexpr int TM = 128, TN = 256, TK = 16;
-constexpr int A_BOX = TM * TK * 4;                 // 8 KB: 128 rows x 64 B
-constexpr int B_BOX = 128 * TK * 4;                // 8 KB: 128 N-rows x 64 B
-constexpr int STAGE = 2 * A_BOX + 2 * (TN / 128) * B_BOX;   // 48 KB
-constexpr int STAGES = 4;
-constexpr int MAX_SEG = 2;       // stages per TMEM segment: 1 (16 K-values) or 2 (32)
+constexpr int TM = 128, TN = 256, TK = 32;
+constexpr int A_BOX = TM * TK * 4;                 // 16 KB: 128 rows x 128 B
+constexpr int B_BOX = 128 * TK * 4;                // 16 KB: 128 N-rows x 128 B
+constexpr int STAGE = 2 * A_BOX + 2 * (TN / 128) * B_BOX;   // 96 KB
+constexpr int STAGES = 2;
 constexpr int THREADS = 320;
 constexpr int SMEM = STAGES * STAGE + 1024 /*align*/ + 256 /*barriers*/;
 constexpr uint32_t TMEM_COLS = 2 * TN;
@@ -56,7 +57,6 @@ struct Prob {
   int lower;         // skip tiles with no entry on or below the diagonal (n - n_lo <= m)
   int vec;           // D rows 16-byte aligned
   uint32_t wait_limit;   // polls of an mbarrier wait before it gives up
-  int seg;               // stages per TMEM segment (1 .. MAX_SEG)
 };
 
 // t-th tile in grouped order: GROUP_M row tiles, all column tiles, then the next group.
@@ -91,7 +91,6 @@ k_gemm3_tf32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CU
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_items = p.ntm * p.ntn;
-  const int nseg = (p.nk + p.seg - 1) / p.seg;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < STAGES; ++i) {
@@ -156,56 +155,39 @@ k_gemm3_tf32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CU
         int tm, tn;
         tile_of(p, w, tm, tn);
         if (!tile_live(p, tm, tn)) continue;
-        for (int sg = 0; sg < nseg && ok; ++sg) {
-          const int s0 = sg * p.seg, s1 = min(s0 + p.seg, p.nk);
+        for (int s = 0; s < p.nk && ok; ++s) {
+          // one stage is one TMEM segment
           if (!tc::mbar_wait(acc_empty + acc, acc_phase ^ 1u, abort_flag, p.wait_limit)) { ok = false; break; }
+          if (!tc::mbar_wait(full + stage, phase, abort_flag, p.wait_limit)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t d = tmem_base + uint32_t(acc * TN);
-          // Both operands K-major in 64-byte rows: 8 K-values = 32 bytes, 8-row groups
-          // 512 bytes apart (the two 128-row B boxes are contiguous).  The segment's
-          // small cross products go first, into its fresh accumulator, and the
-          // hi*hi products after them, so that the accumulator's truncation is
-          // charged mostly at the magnitude of the small sums.  A stage is released
-          // once its hi*hi products are issued.
-          const int st0 = stage;
-          const uint32_t ph0 = phase;
-          for (int s = s0; s < s1 && ok; ++s) {
-            if (!tc::mbar_wait(full + stage, phase, abort_flag, p.wait_limit)) { ok = false; break; }
-            tc::fence_after_sync();
-            const uint8_t* sb = smem + stage * STAGE;
-            const uint8_t* ah = sb;
-            const uint8_t* al = sb + A_BOX;
-            const uint8_t* bh = sb + 2 * A_BOX;
-            const uint8_t* bl = bh + (TN / 128) * B_BOX;
+          // Both operands K-major in 128-byte rows: 8 K-values = 32 bytes, 8-row groups
+          // 1024 bytes apart (the two 128-row B boxes are contiguous).  The small cross
+          // products go first, into the fresh accumulator, and the hi*hi products
+          // after them, so that the accumulator's truncation is charged mostly at the
+          // magnitude of the small sums.
+          const uint8_t* ah = smem + stage * STAGE;
+          const uint8_t* al = ah + A_BOX;
+          const uint8_t* bh = ah + 2 * A_BOX;
+          const uint8_t* bl = bh + (TN / 128) * B_BOX;
 #pragma unroll
-            for (int kk = 0; kk < TK / 8; ++kk) {
-              const uint64_t dah = tc::smem_desc_sw64(ah + kk * 32, 16, 512);
-              const uint64_t dal = tc::smem_desc_sw64(al + kk * 32, 16, 512);
-              const uint64_t dbh = tc::smem_desc_sw64(bh + kk * 32, 16, 512);
-              const uint64_t dbl = tc::smem_desc_sw64(bl + kk * 32, 16, 512);
-              tc::mma_tf32(d, dah, dbl, idesc, (s == s0 && kk == 0) ? 0u : 1u);
-              tc::mma_tf32(d, dal, dbh, idesc, 1u);
-            }
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          for (int kk = 0; kk < TK / 8; ++kk) {
+            const uint64_t dah = tc::smem_desc_sw128(ah + kk * 32, 16, 1024);
+            const uint64_t dal = tc::smem_desc_sw128(al + kk * 32, 16, 1024);
+            const uint64_t dbh = tc::smem_desc_sw128(bh + kk * 32, 16, 1024);
+            const uint64_t dbl = tc::smem_desc_sw128(bl + kk * 32, 16, 1024);
+            tc::mma_tf32(d, dah, dbl, idesc, kk == 0 ? 0u : 1u);
+            tc::mma_tf32(d, dal, dbh, idesc, 1u);
           }
-          if (!ok) break;
-          stage = st0;
-          phase = ph0;
-          for (int s = s0; s < s1; ++s) {
-            const uint8_t* sb = smem + stage * STAGE;
-            const uint8_t* ah = sb;
-            const uint8_t* bh = sb + 2 * A_BOX;
 #pragma unroll
-            for (int kk = 0; kk < TK / 8; ++kk) {
-              const uint64_t dah = tc::smem_desc_sw64(ah + kk * 32, 16, 512);
-              const uint64_t dbh = tc::smem_desc_sw64(bh + kk * 32, 16, 512);
-              tc::mma_tf32(d, dah, dbh, idesc, 1u);
-            }
-            tc::mma_commit(empty + stage);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          for (int kk = 0; kk < TK / 8; ++kk) {
+            const uint64_t dah = tc::smem_desc_sw128(ah + kk * 32, 16, 1024);
+            const uint64_t dbh = tc::smem_desc_sw128(bh + kk * 32, 16, 1024);
+            tc::mma_tf32(d, dah, dbh, idesc, 1u);
           }
-          if (!ok) break;
+          tc::mma_commit(empty + stage);
           tc::mma_commit(acc_full + acc);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
         }
       }
@@ -224,7 +206,7 @@ k_gemm3_tf32(const __grid_constant__ CUtensorMap ahi, const __grid_constant__ CU
       float r[128];
 #pragma unroll
       for (int q = 0; q < 128; ++q) r[q] = 0.f;
-      for (int sg = 0; sg < nseg; ++sg) {
+      for (int s = 0; s < p.nk; ++s) {
         if (!tc::mbar_wait(acc_full + acc, acc_phase, abort_flag, p.wait_limit)) { ok = false; break; }
         tc::fence_after_sync();
 #pragma unroll
@@ -292,7 +274,7 @@ bool encode_k_major(CUtensorMap* m, const float* base, uint64_t ld, uint64_t row
   const cuuint32_t box[2] = {uint32_t(TK), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -301,7 +283,7 @@ bool encode_k_major(CUtensorMap* m, const float* base, uint64_t ld, uint64_t row
 gptq_status gemm3_tf32(cudaStream_t st, float* D, int64_t ldd, int M, int n_lo, int n_hi, int K,
                        const float* Ahi, const float* Alo, int lda, int a_k0, const float* Bhi,
                        const float* Blo, int ldb, int b_rows, int b_k0, bool lower,
-                       int32_t* status, int seg_k) {
+                       int32_t* status) {
   if (M <= 0 || n_hi <= n_lo || K <= 0) return GPTQ_OK;
   // K windows start on 16-byte boundaries (TMA x coordinate) and are whole stages
   if (K % TK || a_k0 % 4 || b_k0 % 4 || a_k0 + K > lda || b_k0 + K > ldb || n_lo < 0 ||
@@ -328,7 +310,6 @@ gptq_status gemm3_tf32(cudaStream_t st, float* D, int64_t ldd, int M, int n_lo, 
   p.lower = lower ? 1 : 0;
   p.vec = ((ldd & 3) == 0 && (reinterpret_cast<uintptr_t>(D) & 15) == 0) ? 1 : 0;
   p.wait_limit = pipeline_wait_limit();
-  p.seg = std::max(1, std::min(MAX_SEG, seg_k / TK));
   int64_t live = int64_t(p.ntm) * p.ntn;
   if (lower) {
     live = 0;

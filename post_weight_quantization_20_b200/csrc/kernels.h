@@ -39,12 +39,11 @@ gptq_status split_tf32_t(cudaStream_t st, const float* U, int C, float* hi, floa
 // segmented fp32 accumulation) for m < M and n in [n_lo, n_hi); A is read from
 // column a_k0 of an M x lda buffer, B from column b_k0 of a b_rows x ldb buffer (both
 // K-major, lda and ldb multiples of 4); lower: only tiles with an entry on or below
-// the diagonal (n_lo must be 0); seg_k: K-values accumulated in TMEM before they are
-// added into registers (16 or 32: shorter is more accurate, longer faster)
+// the diagonal (n_lo must be 0); K, a_k0 and b_k0 multiples of 32, 4 and 4
 gptq_status gemm3_tf32(cudaStream_t st, float* D, int64_t ldd, int M, int n_lo, int n_hi, int K,
                        const float* Ahi, const float* Alo, int lda, int a_k0, const float* Bhi,
                        const float* Blo, int ldb, int b_rows, int b_k0, bool lower,
-                       int32_t* status, int seg_k = 32);
+                       int32_t* status);
 
 // selftest kernels (prepare.cu holds the grid-barrier one, next to the barrier)
 gptq_status selftest_mbarrier(cudaStream_t st, int32_t* status);

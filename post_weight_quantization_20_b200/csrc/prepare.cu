@@ -193,7 +193,7 @@ __global__ void k_sym_full(const float* H, int C, float* S, int lds) {
   }
 }
 
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 k_gather_rows(const float* S, int lds, int C, int Cp, const int32_t* perm, const float* lam,
               float* A) {
   extern __shared__ float srow[];
@@ -205,8 +205,10 @@ k_gather_rows(const float* S, int lds, int C, int Cp, const int32_t* perm, const
   }
   int i = perm[C - 1 - a];
   i = min(max(i, 0), C - 1);
-  const float* src = S + int64_t(i) * lds;
-  for (int b = threadIdx.x; b < C; b += blockDim.x) srow[b] = src[b];
+  // the whole padded row (lds floats, lds % 4 == 0, 16-byte aligned rows) in 16-byte loads
+  const float4* src = reinterpret_cast<const float4*>(S + int64_t(i) * lds);
+  float4* s4 = reinterpret_cast<float4*>(srow);
+  for (int b = threadIdx.x; b < lds / 4; b += blockDim.x) s4[b] = src[b];
   __syncthreads();
   const float l = *lam;
   for (int b = threadIdx.x; b < Cp; b += blockDim.x) {
@@ -837,7 +839,9 @@ gptq_status prepare_run(cudaStream_t st, const float* H, int C, const gptq_confi
     GPTQ_LAUNCH(k_sym_full, tg, tb, 0, st, H, C, L.Bx, Cp);
     // the attribute is the largest row any call stages, so concurrent calls agree
     GPTQ_CUDA(allow_smem(k_gather_rows, GATHER_SMEM_MAX_COLS * 4));
-    GPTQ_LAUNCH(k_gather_rows, Cp, 256, C * 4, st, L.Bx, Cp, C, Cp, perm, L.lam, L.A);
+    // one CTA per row: its source row fills up to 224 KB of shared memory, so 32
+    // warps per CTA keep enough loads and stores in flight
+    GPTQ_LAUNCH(k_gather_rows, Cp, 1024, Cp * 4, st, L.Bx, Cp, C, Cp, perm, L.lam, L.A);
     GPTQ_CUDA(cudaMemsetAsync(L.Bx, 0, size_t(Cp) * Cp * sizeof(float), st));
     GPTQ_LAUNCH(k_unit_diag, (Cp + 255) / 256, 256, 0, st, L.Bx, Cp);
   } else {

@@ -29,9 +29,6 @@ namespace gptq {
 
 constexpr int SW_B = 128;                 // panel width (columns)
 constexpr int SW_B2 = 1024;               // second level of the lazy update (8 panels)
-// K-values per TMEM segment of the panel-level update (16 measured no more accurate
-// at layer level and 4% slower)
-constexpr int SW_PANEL_SEG_K = 32;
 constexpr int SW_ESLOTS = 2 * SW_B2 / SW_B;
 constexpr int SW_LDERR = SW_ESLOTS * SW_B; // row stride of the error buffers
 constexpr int SW_TPR = 8;                 // threads per row
@@ -452,7 +449,7 @@ static gptq_status sweep_lookahead(cudaStream_t st, const QuantLayout& L, int R,
     // transposed split Ut[n][k] = U[k][n]
     if (lvl1)
       err = gemm3_tf32(side, L.Wk, C, R, e1, c1, SW_B, L.Ehi, L.Elo, SW_LDERR, slot * SW_B,
-                       L.Uhi, L.Ulo, C, C, i0, false, status, SW_PANEL_SEG_K);
+                       L.Uhi, L.Ulo, C, C, i0, false, status);
     if (err == GPTQ_OK && lvl2)
       err = gemm3_tf32(side, L.Wk, C, R, e2, C, S_end - S0, L.Ehi, L.Elo, SW_LDERR,
                        ((p / per) % 2) * SW_B2, L.Uhi, L.Ulo, C, C, S0, false, status);

@@ -181,13 +181,6 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(const void* p, uint32_t lbo,
          (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// The same for a 64-byte-swizzled operand (8-row atoms of 512 bytes).
-__device__ __forceinline__ uint64_t smem_desc_sw64(const void* p, uint32_t lbo, uint32_t sbo) {
-  const uint64_t a = smem_u32(p);
-  return ((a >> 4) & 0x3FFFull) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
-         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
-}
-
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
