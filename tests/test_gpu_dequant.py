@@ -71,6 +71,37 @@ def test_dequant_matmul_matches_oracle(R, C, bits, g, M, act, xdt):
     assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / bound)
 
 
+@pytest.mark.parametrize("R,C", [(200, 2112), (70, 640), (129, 4160)])
+@pytest.mark.parametrize("g", [0, 64, 128])
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 11])
+@pytest.mark.parametrize("act", [False, True])
+@pytest.mark.parametrize("xdt", [S.F16, S.BF16])
+def test_dequant_matmul_4bit_shapes(R, C, g, M, act, xdt):
+    """4-bit codes with 16-bit X over group sizes 64 / 128 / per row: the same bound as
+    above, on row counts that are not a multiple of a CTA's rows, column counts that end
+    inside a staged 2048-column chunk with a short last group, and token counts that
+    split into blocks of 8."""
+    codes, scales, zeros, perm, g_idx = _stored(R, C, 4, g, act, R + C + g + M)
+    X = S.gen_activations(M, C, xdt, S.ActSpec(), seed=M + g)
+    packed = o.pack(codes, 4)
+    ref = o.dequant_matmul(S.to_f64(X, xdt), packed, scales, zeros, g_idx, 4)
+    dp = torch.from_numpy(packed.view(np.int32)).to(DEV)
+    dperm = torch.from_numpy(perm).to(DEV)
+    qp = torch.empty(R, G.sweep_words(C, 4), dtype=torch.int32, device=DEV)
+    G.gptq_repack_sweep_order(dp, 4, dperm, qp)
+    Xd = torch.from_numpy(X.view(np.int16) if xdt == S.BF16 else X).to(DEV)
+    if xdt == S.BF16:
+        Xd = Xd.view(torch.bfloat16)
+    Y = torch.full((M, R), float("nan"), device=DEV)
+    G.gptq_dequant_matmul(Xd, qp, torch.from_numpy(scales).to(DEV), torch.from_numpy(zeros).to(DEV),
+                          4, g, dperm if act else None, Y)
+    torch.cuda.synchronize()
+    got = Y.cpu().numpy().astype(np.float64)
+    mag = np.abs(S.to_f64(X, xdt)) @ (scales[:, g_idx] * (codes + zeros[:, g_idx])).T
+    bound = 4 * C * 2.0 ** -24 * mag + 1e-30
+    assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / bound)
+
+
 @pytest.mark.parametrize("R,C", [(300, 2144), (17, 96)])
 @pytest.mark.parametrize("g", [0, 128])
 @pytest.mark.parametrize("M", [1, 2, 3])
