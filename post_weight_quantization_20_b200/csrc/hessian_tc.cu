@@ -2,6 +2,10 @@
 //   H[i][j] += beta * sum_t X[t][i] X[t][j]      (upper-triangle tiles, fp16/bf16 in, fp32 acc)
 // for GPTQ量化算法深度解析 §3.1 step 1.
 //
+// Two forms: on CTA pairs (the second kernel below, 256 x 256 tiles, the default)
+// and on one SM per tile (the first, for a device on which clusters of two cannot
+// be resident).  The one-SM form:
+//
 // Output tile 128 (i) x 256 (j); both operands are read straight from row-major
 // X by TMA as 64-token x 64-column boxes with 128-byte swizzle, which is the
 // MN-major layout tcgen05 consumes (no transpose pass over X).  Per CTA:
